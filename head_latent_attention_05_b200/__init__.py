@@ -1,0 +1,169 @@
+"""Python binding of libmla.so (MLA decode over a paged latent KV cache on B200).
+
+The functions below carry the names of the C ABI in include/mla.h and only marshal arguments:
+torch tensors are passed as raw device pointers with the current CUDA stream, and a non-zero
+status raises MlaError. All computation happens in the CUDA library; there is no fallback.
+If libmla.so has not been built, importing works but every call raises.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libmla.so")
+
+MLA_DTYPE_F32 = 0
+MLA_DTYPE_BF16 = 1
+
+STATUS = {
+    0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
+    3: "MLA_ERR_WORKSPACE_TOO_SMALL", 4: "MLA_ERR_CUDA", 5: "MLA_ERR_DEVICE_TIMEOUT",
+    6: "MLA_ERR_DEVICE_OOB", 7: "MLA_ERR_DEVICE_BAD_LENGTH",
+}
+
+# Every symbol include/mla.h declares (checked by the tests against the built library).
+EXPORTED = (
+    "mla_status_string", "mla_absorb_weights", "mla_append_workspace_size", "mla_append_latent",
+    "mla_decode_workspace_size", "mla_decode", "mla_prefill_ref_workspace_size",
+    "mla_prefill_ref", "mla_get_device_error",
+)
+
+
+class MlaError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)}")
+
+
+class MlaConfig(ctypes.Structure):
+    _fields_ = [
+        ("n_heads", ctypes.c_int32), ("d_model", ctypes.c_int32), ("d_c", ctypes.c_int32),
+        ("d_rope", ctypes.c_int32), ("d_nope", ctypes.c_int32), ("d_v", ctypes.c_int32),
+        ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
+        ("rope_theta", ctypes.c_float),
+    ]
+
+
+def make_config(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size=64, dtype="bf16",
+                softmax_scale=None, rms_eps=1e-6, rope_theta=10000.0) -> MlaConfig:
+    if softmax_scale is None:
+        softmax_scale = 1.0 / math.sqrt(d_nope + d_rope)
+    dt = {"bf16": MLA_DTYPE_BF16, "f32": MLA_DTYPE_F32,
+          torch.bfloat16: MLA_DTYPE_BF16, torch.float32: MLA_DTYPE_F32}[dtype]
+    return MlaConfig(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size, dt,
+                     softmax_scale, rms_eps, rope_theta)
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Load libmla.so from the package directory; raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python head_latent_attention_05_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, SZ, CFG = ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t, ctypes.POINTER(MlaConfig)
+    sig = {
+        "mla_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+        "mla_absorb_weights": (ctypes.c_int, [CFG, P, P, P, P]),
+        "mla_append_workspace_size": (SZ, [CFG, I32]),
+        "mla_append_latent": (ctypes.c_int, [CFG, P, I32, P, P, P, P, P, I32, I32, P, I32, P, SZ, P]),
+        "mla_decode_workspace_size": (SZ, [CFG, I32, I32]),
+        "mla_decode": (ctypes.c_int, [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P, P]),
+        "mla_prefill_ref_workspace_size": (SZ, [CFG, I32, I32]),
+        "mla_prefill_ref": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ, P, P]),
+        "mla_get_device_error": (ctypes.c_int, [P]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype, fn.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def _ptr(t: torch.Tensor):
+    if not t.is_contiguous():
+        raise ValueError("tensors passed to libmla must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _check(code: int, where: str):
+    if code != 0:
+        raise MlaError(code, where)
+
+
+def mla_status_string(code: int) -> str:
+    return load_library().mla_status_string(code).decode()
+
+
+def mla_absorb_weights(cfg: MlaConfig, wkv_b, w_uk_t, w_uv, stream=None):
+    _check(load_library().mla_absorb_weights(ctypes.byref(cfg), _ptr(wkv_b), _ptr(w_uk_t),
+                                             _ptr(w_uv), _stream(stream)), "mla_absorb_weights")
+
+
+def mla_append_workspace_size(cfg: MlaConfig, n_tok: int) -> int:
+    return int(load_library().mla_append_workspace_size(ctypes.byref(cfg), n_tok))
+
+
+def mla_append_latent(cfg: MlaConfig, x, w_dkv, kv_gain, seq_idx, pos, block_table, cache,
+                      workspace, stream=None):
+    batch, max_pages = block_table.shape
+    _check(load_library().mla_append_latent(
+        ctypes.byref(cfg), _ptr(x), x.shape[0], _ptr(w_dkv), _ptr(kv_gain), _ptr(seq_idx),
+        _ptr(pos), _ptr(block_table), batch, max_pages, _ptr(cache), cache.shape[0],
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+        "mla_append_latent")
+
+
+def mla_decode_workspace_size(cfg: MlaConfig, batch: int, tq: int) -> int:
+    return int(load_library().mla_decode_workspace_size(ctypes.byref(cfg), batch, tq))
+
+
+def mla_decode(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv, workspace, out,
+               stream=None):
+    batch, tq = q.shape[0], q.shape[1]
+    _check(load_library().mla_decode(
+        ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), _ptr(w_uk_t), _ptr(w_uv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)), "mla_decode")
+
+
+def mla_prefill_ref_workspace_size(cfg: MlaConfig, batch: int, t_new: int) -> int:
+    return int(load_library().mla_prefill_ref_workspace_size(ctypes.byref(cfg), batch, t_new))
+
+
+def mla_prefill_ref(cfg: MlaConfig, x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens, block_table,
+                    cache, workspace, out, stream=None):
+    batch, t_new = q.shape[0], q.shape[1]
+    _check(load_library().mla_prefill_ref(
+        ctypes.byref(cfg), _ptr(x), _ptr(q), batch, t_new, _ptr(w_dkv), _ptr(kv_gain),
+        _ptr(w_uk_t), _ptr(w_uv), _ptr(seq_lens), _ptr(block_table), block_table.shape[1],
+        _ptr(cache), cache.shape[0], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
+        "mla_prefill_ref")
+
+
+def mla_get_device_error(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the library's device error code."""
+    return int(load_library().mla_get_device_error(_stream(stream)))
+
+
+def workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A 256-byte-aligned byte buffer of at least nbytes (torch's allocator aligns to 512)."""
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)

@@ -1,0 +1,536 @@
+// libmla.so: the C ABI declared in include/mla.h.
+//
+// Host side of every entry point: validate the arguments (nothing is launched on error), carve
+// the caller's workspace, encode TMA descriptors and enqueue the kernels on the caller's
+// stream. No device memory is ever allocated here.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/mla.h"
+#include "common.cuh"
+#include "ptx.cuh"
+#include "simt.cuh"
+#include "tc_decode.cuh"
+#include "tc_gemm.cuh"
+
+using namespace mla;
+
+namespace {
+
+// ------------------------------------------------------------------------------ helpers
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+struct Carve {
+  uint8_t* base;
+  size_t off = 0;
+  explicit Carve(void* b) : base(static_cast<uint8_t*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    T* p = reinterpret_cast<T*>(base == nullptr ? nullptr : base + off);
+    off += align_up(count * sizeof(T));
+    return p;
+  }
+};
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int elem_bytes(const mla_config* c) { return c->dtype == MLA_DTYPE_F32 ? 4 : 2; }
+
+mla_status check_config(const mla_config* c) {
+  if (c == nullptr) return MLA_ERR_INVALID_ARG;
+  if (c->n_heads < 1 || c->d_model < 1 || c->d_c < 1 || c->d_rope < 2 || (c->d_rope & 1) ||
+      c->d_nope < 1 || c->d_v < 1 || c->page_size < 1)
+    return MLA_ERR_INVALID_ARG;
+  if (c->dtype != MLA_DTYPE_F32 && c->dtype != MLA_DTYPE_BF16) return MLA_ERR_INVALID_ARG;
+  if (!(c->softmax_scale > 0.0f) || !std::isfinite(c->softmax_scale)) return MLA_ERR_INVALID_ARG;
+  if (!(c->rms_eps >= 0.0f) || !(c->rope_theta > 0.0f)) return MLA_ERR_INVALID_ARG;
+  // every row must stay 16-byte aligned for vector loads and TMA
+  const int64_t row_bytes = static_cast<int64_t>(c->d_c + c->d_rope) * elem_bytes(c);
+  if (row_bytes % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  return MLA_OK;
+}
+
+// The bf16 decode path: tcgen05 kernels written for DeepSeek-V2 latent shapes.
+bool tc_decode_shape(const mla_config* c) {
+  return c->dtype == MLA_DTYPE_BF16 && c->d_c == ATT_DC && c->d_rope == ATT_DR &&
+         c->page_size == ATT_PAGE && c->d_nope % 64 == 0;
+}
+
+int device_sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+mla_status last_launch_status() {
+  return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault,
+                                         &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// bf16 tensor map with 128-byte swizzle. dims[0] is the contiguous dimension; strides are the
+// byte strides of dims 1.. ; box[0] must be 64 (one 128-byte swizzle row).
+bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+              const uint64_t* strides_bytes, const uint32_t* box) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t d[3], s[2];
+  cuuint32_t bx[3], es[3] = {1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, bx, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Largest dynamic shared memory a kernel asks for: raise its limit once per device.
+template <typename K>
+bool allow_smem(K kernel, int bytes) {
+  if (bytes <= 48 * 1024) return true;
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
+         cudaSuccess;
+}
+
+// ------------------------------------------------------------------ tcgen05 GEMM launcher
+
+int pick_bn(int n) {
+  if (n <= 16) return 16;
+  if (n <= 32) return 32;
+  if (n <= 64) return 64;
+  if (n <= 128) return 128;
+  return 256;
+}
+
+template <int BN, class Epi>
+mla_status launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const GemmShape& shp,
+                          int m_tiles, int Z, const Epi& epi, cudaStream_t st) {
+  auto kern = gemm_tc_kernel<BN, Epi>;
+  constexpr int smem = gemm_smem_bytes<BN>();
+  if (!allow_smem(kern, smem)) return MLA_ERR_CUDA;
+  const dim3 grid(m_tiles, (shp.N + BN - 1) / BN, Z * shp.k_splits);
+  kern<<<grid, 128, smem, st>>>(A, B, shp, epi);
+  return last_launch_status();
+}
+
+template <class Epi>
+mla_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const GemmShape& shp,
+                       int m_tiles, int Z, const Epi& epi, cudaStream_t st) {
+  switch (pick_bn(shp.N)) {
+    case 16: return launch_gemm_bn<16>(A, B, shp, m_tiles, Z, epi, st);
+    case 32: return launch_gemm_bn<32>(A, B, shp, m_tiles, Z, epi, st);
+    case 64: return launch_gemm_bn<64>(A, B, shp, m_tiles, Z, epi, st);
+    case 128: return launch_gemm_bn<128>(A, B, shp, m_tiles, Z, epi, st);
+    default: return launch_gemm_bn<256>(A, B, shp, m_tiles, Z, epi, st);
+  }
+}
+
+// Split-K plan of the append down-projection (identical in the size query and the call).
+struct AppendPlan {
+  int m_tiles, k_chunks, chunks_per_split, k_splits;
+};
+AppendPlan append_plan(const mla_config* c, int n_tok) {
+  AppendPlan p{};
+  const int row = c->d_c + c->d_rope;
+  p.m_tiles = (row + 127) / 128;
+  p.k_chunks = c->d_model / 64;
+  const int n_tiles = (n_tok + 255) / 256;
+  const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
+  int splits = (2 * sms + p.m_tiles * n_tiles - 1) / (p.m_tiles * n_tiles);
+  splits = splits < 1 ? 1 : (splits > p.k_chunks ? p.k_chunks : splits);
+  p.chunks_per_split = (p.k_chunks + splits - 1) / splits;
+  p.k_splits = (p.k_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
+  return p;
+}
+
+bool tc_append_shape(const mla_config* c) {
+  return c->dtype == MLA_DTYPE_BF16 && c->d_model % 64 == 0;
+}
+
+// ------------------------------------------------------------------ decode workspace layout
+
+struct DecodeLayout {
+  int P, n_mt, R, U, max_segs;
+  int32_t *unit_tiles, *unit_seg, *pair_seg;
+  AttnSeg* segs;
+  __nv_bfloat16 *qhat, *o_lat;
+  float *o_part, *lse;
+  size_t bytes;
+};
+
+DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
+  DecodeLayout L{};
+  const int sms = device_sm_count();
+  L.P = (sms >= 2 ? sms : 2) / 2;
+  L.R = Tq * c->n_heads;
+  L.n_mt = (L.R + 127) / 128;
+  L.U = B * L.n_mt;
+  L.max_segs = L.U + L.P;
+  Carve cv(ws);
+  L.unit_tiles = cv.take<int32_t>(L.U);
+  L.unit_seg = cv.take<int32_t>(L.U + 1);
+  L.pair_seg = cv.take<int32_t>(L.P + 1);
+  L.segs = cv.take<AttnSeg>(L.max_segs);
+  L.qhat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_ROW);
+  L.o_lat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_DC);
+  L.o_part = cv.take<float>(static_cast<size_t>(L.max_segs) * 128 * ATT_DC);
+  L.lse = cv.take<float>(static_cast<size_t>(L.max_segs) * 128);
+  L.bytes = cv.off;
+  return L;
+}
+
+struct SimtLayout {
+  float *qhat, *o_lat, *kv;
+  int32_t *seq_idx, *pos;
+  size_t bytes;
+};
+
+SimtLayout simt_layout(const mla_config* c, int64_t rows, int64_t n_append_tok, void* ws) {
+  SimtLayout L{};
+  Carve cv(ws);
+  L.kv = cv.take<float>(static_cast<size_t>(n_append_tok) * (c->d_c + c->d_rope));
+  L.seq_idx = cv.take<int32_t>(static_cast<size_t>(n_append_tok));
+  L.pos = cv.take<int32_t>(static_cast<size_t>(n_append_tok));
+  L.qhat = cv.take<float>(static_cast<size_t>(rows) * (c->d_c + c->d_rope));
+  L.o_lat = cv.take<float>(static_cast<size_t>(rows) * c->d_c);
+  L.bytes = cv.off;
+  return L;
+}
+
+// -------------------------------------------------------------------- SIMT decode (any T)
+
+template <typename T>
+mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const void* cache,
+                       int num_pages, const int32_t* block_table, int max_pages,
+                       const int32_t* seq_lens, const void* w_uk_t, const void* w_uv,
+                       const SimtLayout& L, void* out, cudaStream_t st) {
+  const int rows = B * Tq * c->n_heads;
+  const int row = c->d_c + c->d_rope;
+  const int max_pos = max_pages * c->page_size;
+  qabs_simt_kernel<T><<<rows, 256, (c->d_nope + c->d_rope) * sizeof(float), st>>>(
+      static_cast<const T*>(q), static_cast<const T*>(w_uk_t), seq_lens, L.qhat, c->n_heads,
+      Tq, c->d_c, c->d_rope, c->d_nope, max_pos, c->rope_theta);
+  const int attn_smem = (row + c->d_c) * static_cast<int>(sizeof(float));
+  if (!allow_smem(attn_simt_kernel<T>, attn_smem)) return MLA_ERR_CUDA;
+  attn_simt_kernel<T><<<rows, 256, attn_smem, st>>>(
+      L.qhat, static_cast<const T*>(cache), block_table, seq_lens, L.o_lat, c->n_heads, Tq,
+      c->d_c, c->d_rope, max_pages, num_pages, c->page_size, c->softmax_scale);
+  outproj_simt_kernel<T><<<rows, 256, c->d_c * sizeof(float), st>>>(
+      L.o_lat, static_cast<const T*>(w_uv), static_cast<T*>(out), c->n_heads, c->d_c, c->d_v);
+  return last_launch_status();
+}
+
+template <typename T>
+mla_status simt_append(const mla_config* c, const void* x, int n_tok, const void* w_dkv,
+                       const void* kv_gain, const int32_t* seq_idx, const int32_t* pos,
+                       const int32_t* block_table, int batch, int max_pages, void* cache,
+                       int num_pages, float* kv, cudaStream_t st) {
+  const int row = c->d_c + c->d_rope;
+  const dim3 g1((row + 7) / 8, n_tok);
+  linear_rows_kernel<T><<<g1, 256, 0, st>>>(static_cast<const T*>(x),
+                                            static_cast<const T*>(w_dkv), kv, n_tok, row,
+                                            c->d_model);
+  append_finish_kernel<T><<<n_tok, 256, row * sizeof(float), st>>>(
+      kv, 1, n_tok, static_cast<const T*>(kv_gain), seq_idx, pos, block_table, batch,
+      max_pages, static_cast<T*>(cache), num_pages, c->page_size, c->d_c, c->d_rope,
+      c->rms_eps, c->rope_theta);
+  return last_launch_status();
+}
+
+__global__ void prefill_positions_kernel(const int32_t* __restrict__ seq_lens, int t_new,
+                                         int n_tok, int32_t* __restrict__ seq_idx,
+                                         int32_t* __restrict__ pos) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n_tok) return;
+  const int b = i / t_new, t = i % t_new;
+  seq_idx[i] = b;
+  pos[i] = seq_lens[b] - t_new + t;  // out-of-range values are caught by the append kernel
+}
+
+}  // namespace
+
+// ====================================================================== exported functions
+
+extern "C" {
+
+const char* mla_status_string(mla_status s) {
+  switch (s) {
+    case MLA_OK: return "MLA_OK";
+    case MLA_ERR_INVALID_ARG: return "MLA_ERR_INVALID_ARG";
+    case MLA_ERR_UNSUPPORTED: return "MLA_ERR_UNSUPPORTED";
+    case MLA_ERR_WORKSPACE_TOO_SMALL: return "MLA_ERR_WORKSPACE_TOO_SMALL";
+    case MLA_ERR_CUDA: return "MLA_ERR_CUDA";
+    case MLA_ERR_DEVICE_TIMEOUT: return "MLA_ERR_DEVICE_TIMEOUT";
+    case MLA_ERR_DEVICE_OOB: return "MLA_ERR_DEVICE_OOB";
+    case MLA_ERR_DEVICE_BAD_LENGTH: return "MLA_ERR_DEVICE_BAD_LENGTH";
+  }
+  return "MLA_ERR_UNKNOWN";
+}
+
+mla_status mla_absorb_weights(const mla_config* cfg, const void* wkv_b, void* w_uk_t,
+                              void* w_uv, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (wkv_b == nullptr || w_uk_t == nullptr || w_uv == nullptr) return MLA_ERR_INVALID_ARG;
+  if (!aligned16(wkv_b) || !aligned16(w_uk_t) || !aligned16(w_uv)) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t total = static_cast<int64_t>(cfg->n_heads) * (cfg->d_nope + cfg->d_v) * cfg->d_c;
+  const int blocks = static_cast<int>((total + 255) / 256 < 65535 * 8 ? (total + 255) / 256 : 65535 * 8);
+  if (cfg->dtype == MLA_DTYPE_F32)
+    absorb_kernel<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(wkv_b),
+                                                 static_cast<float*>(w_uk_t),
+                                                 static_cast<float*>(w_uv), cfg->n_heads,
+                                                 cfg->d_c, cfg->d_nope, cfg->d_v);
+  else
+    absorb_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(wkv_b), static_cast<__nv_bfloat16*>(w_uk_t),
+        static_cast<__nv_bfloat16*>(w_uv), cfg->n_heads, cfg->d_c, cfg->d_nope, cfg->d_v);
+  return last_launch_status();
+}
+
+size_t mla_append_workspace_size(const mla_config* cfg, int32_t n_tok) {
+  if (check_config(cfg) != MLA_OK || n_tok < 1) return 0;
+  const size_t row = static_cast<size_t>(cfg->d_c + cfg->d_rope);
+  if (cfg->dtype == MLA_DTYPE_BF16) {
+    if (!tc_append_shape(cfg)) return 0;
+    const AppendPlan p = append_plan(cfg, n_tok);
+    return align_up(static_cast<size_t>(p.k_splits) * n_tok * row * sizeof(float));
+  }
+  return align_up(static_cast<size_t>(n_tok) * row * sizeof(float));
+}
+
+mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok,
+                             const void* w_dkv, const void* kv_gain, const int32_t* seq_idx,
+                             const int32_t* pos, const int32_t* block_table, int32_t batch,
+                             int32_t max_pages, void* cache, int32_t num_pages, void* workspace,
+                             size_t ws_bytes, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (n_tok < 1 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_dkv, kv_gain, seq_idx, pos, block_table, cache, workspace};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype == MLA_DTYPE_BF16 && !tc_append_shape(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (ws_bytes < mla_append_workspace_size(cfg, n_tok)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int row = cfg->d_c + cfg->d_rope;
+  if (cfg->dtype == MLA_DTYPE_F32)
+    return simt_append<float>(cfg, x, n_tok, w_dkv, kv_gain, seq_idx, pos, block_table, batch,
+                              max_pages, cache, num_pages, static_cast<float*>(workspace), st);
+
+  // bf16: tcgen05 split-K GEMM kv = x · w_dkvᵀ, then norm / RoPE / scatter per token
+  const AppendPlan ap = append_plan(cfg, n_tok);
+  CUtensorMap mA, mB;
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(cfg->d_model), static_cast<uint64_t>(row), 1};
+    const uint64_t strides[2] = {static_cast<uint64_t>(cfg->d_model) * 2,
+                                 static_cast<uint64_t>(cfg->d_model) * 2 * row};
+    const uint32_t box[3] = {64, 128, 1};
+    if (!make_map(&mA, w_dkv, 3, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[3] = {static_cast<uint64_t>(cfg->d_model), 1, static_cast<uint64_t>(n_tok)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(cfg->d_model) * 2,
+                                 static_cast<uint64_t>(cfg->d_model) * 2};
+    const uint32_t box[3] = {64, 1, static_cast<uint32_t>(pick_bn(n_tok))};
+    if (!make_map(&mB, x, 3, dims, strides, box)) return MLA_ERR_CUDA;
+  }
+  float* partial = static_cast<float*>(workspace);
+  GemmShape shp{row, n_tok, ap.k_chunks, ap.chunks_per_split, ap.k_splits, 0};
+  EpiSplitK epi{partial, n_tok, row};
+  mla_status s = launch_gemm(mA, mB, shp, ap.m_tiles, 1, epi, st);
+  if (s != MLA_OK) return s;
+  append_finish_kernel<__nv_bfloat16><<<n_tok, 256, row * sizeof(float), st>>>(
+      partial, ap.k_splits, n_tok, static_cast<const __nv_bfloat16*>(kv_gain), seq_idx, pos,
+      block_table, batch, max_pages, static_cast<__nv_bfloat16*>(cache), num_pages,
+      cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps, cfg->rope_theta);
+  return last_launch_status();
+}
+
+size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq) {
+  if (check_config(cfg) != MLA_OK || batch < 1 || tq < 1) return 0;
+  if (cfg->dtype == MLA_DTYPE_BF16) {
+    if (!tc_decode_shape(cfg)) return 0;
+    return decode_layout_tc(cfg, batch, tq, nullptr).bytes;
+  }
+  return simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, nullptr).bytes;
+}
+
+mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                      const void* cache, int32_t num_pages, const int32_t* block_table,
+                      int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                      const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                      void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (batch < 1 || tq < 1 || num_pages < 1 || max_pages < 1) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, cache, block_table, seq_lens, w_uk_t, w_uv, workspace, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(max_pages) * cfg->page_size > (1 << 30)) return MLA_ERR_INVALID_ARG;
+  if (cfg->dtype == MLA_DTYPE_BF16 && !tc_decode_shape(cfg)) return MLA_ERR_UNSUPPORTED;
+  if (ws_bytes < mla_decode_workspace_size(cfg, batch, tq)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  if (cfg->dtype == MLA_DTYPE_F32) {
+    const SimtLayout L = simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, workspace);
+    return simt_decode<float>(cfg, q, batch, tq, cache, num_pages, block_table, max_pages,
+                              seq_lens, w_uk_t, w_uv, L, out, st);
+  }
+
+  const DecodeLayout L = decode_layout_tc(cfg, batch, tq, workspace);
+  const int H = cfg->n_heads;
+  const int n_q = batch * tq;                 // query tokens
+  const int max_pos = max_pages * ATT_PAGE;
+  const int qrow = cfg->d_nope + cfg->d_rope;
+
+  // (1) plan the split-KV work list on the device
+  PlanParams pp{seq_lens, batch, tq, L.n_mt, max_pos, L.P, L.max_segs,
+                L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
+  attn_plan_kernel<<<1, 1024, 0, st>>>(pp);
+
+  // (2) Q̂ = [q_nope · W_UK | RoPE(q_rope)]
+  {
+    CUtensorMap mA, mB;
+    const uint64_t da[3] = {static_cast<uint64_t>(cfg->d_nope), ATT_DC, static_cast<uint64_t>(H)};
+    const uint64_t sa[2] = {static_cast<uint64_t>(cfg->d_nope) * 2,
+                            static_cast<uint64_t>(cfg->d_nope) * 2 * ATT_DC};
+    const uint32_t ba[3] = {64, 128, 1};
+    const uint64_t db[3] = {static_cast<uint64_t>(qrow), static_cast<uint64_t>(H),
+                            static_cast<uint64_t>(n_q)};
+    const uint64_t sb[2] = {static_cast<uint64_t>(qrow) * 2, static_cast<uint64_t>(qrow) * 2 * H};
+    const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(pick_bn(n_q))};
+    if (!make_map(&mA, w_uk_t, 3, da, sa, ba) || !make_map(&mB, q, 3, db, sb, bb))
+      return MLA_ERR_CUDA;
+    GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1};
+    EpiQhat epi{L.qhat, static_cast<const __nv_bfloat16*>(q), seq_lens, H, tq, ATT_DC, ATT_DR,
+                cfg->d_nope, n_q, max_pos, cfg->rope_theta};
+    const mla_status s = launch_gemm(mA, mB, shp, ATT_DC / 128, H, epi, st);
+    if (s != MLA_OK) return s;
+  }
+
+  // (3) fused latent attention, one partial per segment
+  {
+    CUtensorMap mc, mq;
+    const uint64_t dc[2] = {ATT_ROW, static_cast<uint64_t>(num_pages) * ATT_PAGE};
+    const uint64_t sc[1] = {ATT_ROW * 2};
+    const uint32_t bc[2] = {64, ATT_PAGE};
+    const uint64_t dq[2] = {ATT_ROW, static_cast<uint64_t>(batch) * L.R};
+    const uint32_t bq[2] = {64, 128};
+    if (!make_map(&mc, cache, 2, dc, sc, bc) || !make_map(&mq, L.qhat, 2, dq, sc, bq))
+      return MLA_ERR_CUDA;
+    AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
+                  max_pages, num_pages, H, tq, L.R, L.n_mt,
+                  cfg->softmax_scale * 1.4426950408889634f};
+    if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
+    mla_decode_attn_kernel<<<2 * L.P, ATT_THREADS, ATT_SMEM_BYTES, st>>>(mc, mq, ap);
+    const mla_status s = last_launch_status();
+    if (s != MLA_OK) return s;
+  }
+
+  // (4) merge split partials -> o_lat (bf16)
+  {
+    const int rows = batch * L.R;
+    attn_combine_kernel<<<(rows + 7) / 8, 256, 0, st>>>(L.o_part, L.lse, L.unit_seg, L.o_lat,
+                                                        rows, L.R, L.n_mt);
+    const mla_status s = last_launch_status();
+    if (s != MLA_OK) return s;
+  }
+
+  // (5) out = o_lat · W_UVᵀ per head
+  {
+    CUtensorMap mA, mB;
+    const uint64_t da[3] = {ATT_DC, static_cast<uint64_t>(cfg->d_v), static_cast<uint64_t>(H)};
+    const uint64_t sa[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * cfg->d_v};
+    const uint32_t ba[3] = {64, 128, 1};
+    const uint64_t db[3] = {ATT_DC, static_cast<uint64_t>(H), static_cast<uint64_t>(n_q)};
+    const uint64_t sb[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * H};
+    const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(pick_bn(n_q))};
+    if (!make_map(&mA, w_uv, 3, da, sa, ba) || !make_map(&mB, L.o_lat, 3, db, sb, bb))
+      return MLA_ERR_CUDA;
+    GemmShape shp{cfg->d_v, n_q, ATT_DC / 64, ATT_DC / 64, 1, 1};
+    EpiOut epi{static_cast<__nv_bfloat16*>(out), H, cfg->d_v};
+    return launch_gemm(mA, mB, shp, (cfg->d_v + 127) / 128, H, epi, st);
+  }
+}
+
+size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new) {
+  if (check_config(cfg) != MLA_OK || batch < 1 || t_new < 1) return 0;
+  const int64_t n = static_cast<int64_t>(batch) * t_new;
+  return simt_layout(cfg, n * cfg->n_heads, n, nullptr).bytes;
+}
+
+mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, int32_t batch,
+                           int32_t t_new, const void* w_dkv, const void* kv_gain,
+                           const void* w_uk_t, const void* w_uv, const int32_t* seq_lens,
+                           const int32_t* block_table, int32_t max_pages, void* cache,
+                           int32_t num_pages, void* workspace, size_t ws_bytes, void* out,
+                           void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (batch < 1 || t_new < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens, block_table, cache,
+                        workspace, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < mla_prefill_ref_workspace_size(cfg, batch, t_new))
+    return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n = batch * t_new;
+  const SimtLayout L = simt_layout(cfg, static_cast<int64_t>(n) * cfg->n_heads, n, workspace);
+  prefill_positions_kernel<<<(n + 255) / 256, 256, 0, st>>>(seq_lens, t_new, n, L.seq_idx, L.pos);
+  mla_status s;
+  if (cfg->dtype == MLA_DTYPE_F32) {
+    s = simt_append<float>(cfg, x, n, w_dkv, kv_gain, L.seq_idx, L.pos, block_table, batch,
+                           max_pages, cache, num_pages, L.kv, st);
+    if (s != MLA_OK) return s;
+    return simt_decode<float>(cfg, q, batch, t_new, cache, num_pages, block_table, max_pages,
+                              seq_lens, w_uk_t, w_uv, L, out, st);
+  }
+  s = simt_append<__nv_bfloat16>(cfg, x, n, w_dkv, kv_gain, L.seq_idx, L.pos, block_table,
+                                 batch, max_pages, cache, num_pages, L.kv, st);
+  if (s != MLA_OK) return s;
+  return simt_decode<__nv_bfloat16>(cfg, q, batch, t_new, cache, num_pages, block_table,
+                                    max_pages, seq_lens, w_uk_t, w_uv, L, out, st);
+}
+
+mla_status mla_get_device_error(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_error, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int)) != cudaSuccess) return MLA_ERR_CUDA;
+  }
+  return static_cast<mla_status>(v);
+}
+
+}  // extern "C"

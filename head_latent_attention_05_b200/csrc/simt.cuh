@@ -1,0 +1,247 @@
+// CUDA-core kernels (fp32 arithmetic, any shape, fp32 or bf16 storage).
+//
+// They implement the fp32 decode path (q absorption, attention, value projection) and the
+// reference prefill path, plus the append step for shapes the tensor-core path does not take
+// and the bit-exact weight split. Each block works on one row (a token, or one (token, head)
+// query) and is written for clarity and coalesced loads rather than peak throughput.
+#pragma once
+
+#include "common.cuh"
+
+namespace mla {
+
+// --------------------------------------------------------------- a0: absorbed weight packs
+// w_uk_t[h][c][n] = wkv_b[h*(dn+dv)+n][c];  w_uv[h][v][c] = wkv_b[h*(dn+dv)+dn+v][c].
+template <typename T>
+__global__ void absorb_kernel(const T* __restrict__ wkv_b, T* __restrict__ w_uk_t,
+                              T* __restrict__ w_uv, int H, int d_c, int d_nope, int d_v) {
+  const int64_t per_head = static_cast<int64_t>(d_nope + d_v) * d_c;
+  const int64_t total = per_head * H;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int h = static_cast<int>(i / per_head);
+    const int64_t rem = i - h * per_head;
+    if (rem < static_cast<int64_t>(d_c) * d_nope) {
+      // output index inside w_uk_t[h]: (c, n), n fastest
+      const int c = static_cast<int>(rem / d_nope), n = static_cast<int>(rem % d_nope);
+      w_uk_t[static_cast<int64_t>(h) * d_c * d_nope + rem] =
+          wkv_b[(static_cast<int64_t>(h) * (d_nope + d_v) + n) * d_c + c];
+    } else {
+      const int64_t r2 = rem - static_cast<int64_t>(d_c) * d_nope;  // (v, c), c fastest
+      const int v = static_cast<int>(r2 / d_c), c = static_cast<int>(r2 % d_c);
+      w_uv[static_cast<int64_t>(h) * d_v * d_c + r2] =
+          wkv_b[(static_cast<int64_t>(h) * (d_nope + d_v) + d_nope + v) * d_c + c];
+    }
+  }
+}
+
+// ------------------------------------------------------------------------ a1: append (SIMT)
+// kv[n][f] = sum_k x[n][k] * w[f][k] in fp32. One warp per output feature, 8 warps per block.
+template <typename T>
+__global__ void __launch_bounds__(256)
+linear_rows_kernel(const T* __restrict__ x, const T* __restrict__ w, float* __restrict__ out,
+                   int n_tok, int F, int K) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int f = blockIdx.x * 8 + warp;
+  const int n = blockIdx.y;
+  if (f >= F || n >= n_tok) return;
+  const T* xr = x + static_cast<int64_t>(n) * K;
+  const T* wr = w + static_cast<int64_t>(f) * K;
+  float acc = 0.0f;
+  for (int k = lane; k < K; k += 32) acc = fmaf(Elem<T>::to_f(xr[k]), Elem<T>::to_f(wr[k]), acc);
+  acc = warp_sum(acc);
+  if (lane == 0) out[static_cast<int64_t>(n) * F + f] = acc;
+}
+
+// Resolve the cache row of (sequence b, position p). Returns nullptr (and records the error)
+// when the sequence index, the position or the page id is out of range.
+template <typename T>
+__device__ __forceinline__ T* cache_row(T* cache, const int32_t* block_table, int b, int p,
+                                        int batch, int max_pages, int num_pages,
+                                        int page_size, int row) {
+  if (b < 0 || b >= batch || p < 0 || p / page_size >= max_pages) return nullptr;
+  const int page = block_table[static_cast<int64_t>(b) * max_pages + p / page_size];
+  if (page < 0 || page >= num_pages) return nullptr;
+  return cache + (static_cast<int64_t>(page) * page_size + p % page_size) * row;
+}
+
+// Per token: RMSNorm over c_KV, RoPE on k_R at the token's position, one rounding to the
+// cache type, scatter to its page slot. kv holds n_splits partial sums [n_splits][n_tok][row],
+// added in a fixed order.
+template <typename T>
+__global__ void __launch_bounds__(256)
+append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
+                     const T* __restrict__ kv_gain, const int32_t* __restrict__ seq_idx,
+                     const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table,
+                     int batch, int max_pages, T* __restrict__ cache, int num_pages,
+                     int page_size, int d_c, int d_r, float eps, float theta) {
+  __shared__ float red[32];
+  extern __shared__ float row_s[];  // [d_c + d_r]
+  const int i = blockIdx.x;
+  const int row = d_c + d_r;
+  const int b = seq_idx[i], p = pos[i];
+  T* dst = cache_row(cache, block_table, b, p, batch, max_pages, num_pages, page_size, row);
+  if (dst == nullptr) {
+    if (threadIdx.x == 0) record_error(MLA_ERR_DEVICE_OOB);
+    return;
+  }
+  float ss = 0.0f;
+  for (int f = threadIdx.x; f < row; f += blockDim.x) {
+    float v = 0.0f;
+    for (int s = 0; s < n_splits; ++s) v += kv[(static_cast<int64_t>(s) * n_tok + i) * row + f];
+    row_s[f] = v;
+    if (f < d_c) ss = fmaf(v, v, ss);
+  }
+  ss = block_sum(ss, red);  // also orders the row_s writes before the reads below
+  const float rstd = 1.0f / sqrtf(ss / static_cast<float>(d_c) + eps);
+  for (int f = threadIdx.x; f < d_c; f += blockDim.x)
+    dst[f] = Elem<T>::from_f(row_s[f] * rstd * Elem<T>::to_f(kv_gain[f]));
+  for (int pr = threadIdx.x; pr < d_r / 2; pr += blockDim.x) {
+    float ox, oy;
+    rope_pair(row_s[d_c + 2 * pr], row_s[d_c + 2 * pr + 1], pr, d_r, p, theta, &ox, &oy);
+    dst[d_c + 2 * pr] = Elem<T>::from_f(ox);
+    dst[d_c + 2 * pr + 1] = Elem<T>::from_f(oy);
+  }
+}
+
+// ---------------------------------------------------- decode on CUDA cores (fp32 arithmetic)
+// Query rows are r = (b*Tq + t)*H + h. The length of sequence b must lie in [Tq, max_pos].
+__device__ __forceinline__ bool length_ok(int L, int Tq, int max_pos) {
+  return L >= Tq && L <= max_pos;
+}
+
+// qhat[r] = [ q_nope·W_UK[h] (d_c) | RoPE(q_rope, L_b - Tq + t) (d_r) ] in fp32.
+template <typename T>
+__global__ void __launch_bounds__(256)
+qabs_simt_kernel(const T* __restrict__ q, const T* __restrict__ w_uk_t,
+                 const int32_t* __restrict__ seq_lens, float* __restrict__ qhat, int H, int Tq,
+                 int d_c, int d_r, int d_nope, int max_pos, float theta) {
+  extern __shared__ float qs[];  // [d_nope + d_r]
+  const int r = blockIdx.x;
+  const int h = r % H, t = (r / H) % Tq, b = r / (H * Tq);
+  const int L = seq_lens[b];
+  const bool ok = length_ok(L, Tq, max_pos);
+  const T* qr = q + static_cast<int64_t>(r) * (d_nope + d_r);
+  float* out = qhat + static_cast<int64_t>(r) * (d_c + d_r);
+  for (int i = threadIdx.x; i < d_nope + d_r; i += blockDim.x) qs[i] = Elem<T>::to_f(qr[i]);
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const T* wh = w_uk_t + static_cast<int64_t>(h) * d_c * d_nope;
+  for (int c = warp; c < d_c; c += nw) {
+    float acc = 0.0f;
+    for (int n = lane; n < d_nope; n += 32)
+      acc = fmaf(qs[n], Elem<T>::to_f(wh[static_cast<int64_t>(c) * d_nope + n]), acc);
+    acc = warp_sum(acc);
+    if (lane == 0) out[c] = ok ? acc : 0.0f;
+  }
+  const int p = L - Tq + t;
+  for (int pr = threadIdx.x; pr < d_r / 2; pr += blockDim.x) {
+    float ox = 0.0f, oy = 0.0f;
+    if (ok) rope_pair(qs[d_nope + 2 * pr], qs[d_nope + 2 * pr + 1], pr, d_r, p, theta, &ox, &oy);
+    out[d_c + 2 * pr] = ox;
+    out[d_c + 2 * pr + 1] = oy;
+  }
+}
+
+// One block per query row: online softmax over chunks of 256 keys.
+//   s_j = scale * qhat · cache_row_j  (all d_c + d_r dims),  j <= L_b - Tq + t
+//   o_lat = sum_j softmax(s)_j * cache_row_j[:d_c]
+template <typename T>
+__global__ void __launch_bounds__(256)
+attn_simt_kernel(const float* __restrict__ qhat, const T* __restrict__ cache,
+                 const int32_t* __restrict__ block_table, const int32_t* __restrict__ seq_lens,
+                 float* __restrict__ o_lat, int H, int Tq, int d_c, int d_r, int max_pages,
+                 int num_pages, int page_size, float scale) {
+  constexpr int CH = 256;
+  __shared__ float red[32];
+  __shared__ float p_s[CH];
+  __shared__ const T* rows_s[CH];
+  extern __shared__ float dyn[];  // qs [d_c + d_r] | acc [d_c]
+  const int row = d_c + d_r;
+  float* qs = dyn;
+  float* acc = dyn + row;
+  const int r = blockIdx.x;
+  const int t = (r / H) % Tq, b = r / (H * Tq);
+  const int L = seq_lens[b];
+  float* out = o_lat + static_cast<int64_t>(r) * d_c;
+  if (!length_ok(L, Tq, max_pages * page_size)) {
+    for (int c = threadIdx.x; c < d_c; c += blockDim.x) out[c] = 0.0f;
+    if (threadIdx.x == 0 && (r % H) == 0 && t == 0) record_error(MLA_ERR_DEVICE_BAD_LENGTH);
+    return;
+  }
+  const int n_keys = L - Tq + t + 1;
+  for (int i = threadIdx.x; i < row; i += blockDim.x) qs[i] = qhat[static_cast<int64_t>(r) * row + i];
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) acc[c] = 0.0f;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  float m = -INFINITY, l = 0.0f;
+  bool oob = false;
+  for (int j0 = 0; j0 < n_keys; j0 += CH) {
+    const int cnt = min(CH, n_keys - j0);
+    for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) {
+      const int j = j0 + jj;
+      const int page = block_table[static_cast<int64_t>(b) * max_pages + j / page_size];
+      const bool bad = page < 0 || page >= num_pages;
+      oob |= bad;
+      rows_s[jj] = bad ? nullptr : cache + (static_cast<int64_t>(page) * page_size + j % page_size) * row;
+    }
+    __syncthreads();
+    for (int jj = warp; jj < cnt; jj += nw) {
+      const T* cr = rows_s[jj];
+      float s = 0.0f;
+      if (cr != nullptr)
+        for (int i = lane; i < row; i += 32) s = fmaf(qs[i], Elem<T>::to_f(cr[i]), s);
+      s = warp_sum(s);
+      if (lane == 0) p_s[jj] = (cr != nullptr) ? s * scale : -INFINITY;
+    }
+    __syncthreads();
+    float cm = -INFINITY;
+    for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) cm = fmaxf(cm, p_s[jj]);
+    cm = block_max(cm, red);
+    const float m_new = fmaxf(m, cm);
+    const float base = (m_new == -INFINITY) ? 0.0f : m_new;
+    const float factor = (m == -INFINITY) ? 0.0f : expf(m - base);
+    float ps = 0.0f;
+    for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) {
+      const float e = expf(p_s[jj] - base);
+      p_s[jj] = e;
+      ps += e;
+    }
+    ps = block_sum(ps, red);  // also publishes p_s
+    l = l * factor + ps;
+    m = m_new;
+    for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
+      float a = acc[c] * factor;
+      for (int jj = 0; jj < cnt; ++jj) {
+        const T* cr = rows_s[jj];
+        if (cr != nullptr) a = fmaf(p_s[jj], Elem<T>::to_f(cr[c]), a);
+      }
+      acc[c] = a;
+    }
+    __syncthreads();
+  }
+  if (oob) record_error(MLA_ERR_DEVICE_OOB);
+  const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) out[c] = acc[c] * inv;
+}
+
+// out[r][v] = sum_c o_lat[r][c] * w_uv[h][v][c]. One warp per output column v.
+template <typename T>
+__global__ void __launch_bounds__(256)
+outproj_simt_kernel(const float* __restrict__ o_lat, const T* __restrict__ w_uv,
+                    T* __restrict__ out, int H, int d_c, int d_v) {
+  extern __shared__ float os[];  // [d_c]
+  const int r = blockIdx.x, h = r % H;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) os[c] = o_lat[static_cast<int64_t>(r) * d_c + c];
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
+  const T* wh = w_uv + static_cast<int64_t>(h) * d_v * d_c;
+  for (int v = warp; v < d_v; v += nw) {
+    float a = 0.0f;
+    for (int c = lane; c < d_c; c += 32) a = fmaf(os[c], Elem<T>::to_f(wh[static_cast<int64_t>(v) * d_c + c]), a);
+    a = warp_sum(a);
+    if (lane == 0) out[static_cast<int64_t>(r) * d_v + v] = Elem<T>::from_f(a);
+  }
+}
+
+}  // namespace mla

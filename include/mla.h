@@ -1,0 +1,183 @@
+/*
+ * mla.h — C ABI of libmla.so: Multi-head Latent Attention (MLA) decode over a paged latent
+ * KV cache on NVIDIA B200 (sm_100a).
+ *
+ * What is computed. Each cached token stores one row [c_KV (d_c) | k_R (d_rope)] shared by all
+ * heads (「论文复现工坊 No.4 从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §1: the cache holds
+ * (d_c + d_R) elements per token). Decoding uses the absorbed form (same page, §4; and
+ * 「淺析DeepSeek多頭潛在注意力機制（MLA）」, section "MLA的數學原理"): per head h
+ *     q_lat = q_nope · W_UK[h]                       (d_nope -> d_c)
+ *     s_j   = (q_lat · c_j + RoPE(q_rope, p) · k_R,j) · softmax_scale
+ *     P     = softmax_j(s),   o_lat = Σ_j P_j c_j,   out = o_lat · W_UV[h]ᵀ   (d_c -> d_v)
+ * which equals the page's expanded module (§2 of the first page) up to rounding.
+ *
+ * Conventions for every call:
+ *   - Tensors are dense, row-major, and live in device memory unless stated otherwise. The
+ *     element type of every floating-point tensor is cfg->dtype (fp32 or bf16). Index tensors
+ *     are int32.
+ *   - The caller owns every buffer. The library never allocates or frees device memory and
+ *     keeps no state between calls other than one device-side error word (see
+ *     mla_get_device_error).
+ *   - Device pointers must be 16-byte aligned.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are asynchronous;
+ *     they enqueue kernels on `stream` and return. Arguments are validated on the host first:
+ *     on any error the call returns a non-zero mla_status and enqueues nothing.
+ *   - Errors that only the device can see (a page id outside the pool, a sequence length out
+ *     of range, a stalled pipeline) are recorded in the device error word; the affected
+ *     outputs are zero-filled, no memory outside the given buffers is touched, and the next
+ *     mla_get_device_error call reports the first such error.
+ *   - Calls that share a workspace or a cache must not overlap on the GPU (use one stream).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,          /* null/unaligned pointer, bad size, inconsistent config  */
+  MLA_ERR_UNSUPPORTED = 2,          /* valid config this build has no kernel for             */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below the matching *_workspace_size()         */
+  MLA_ERR_CUDA = 4,                 /* a CUDA runtime/driver call failed                      */
+  MLA_ERR_DEVICE_TIMEOUT = 5,       /* a kernel's bounded wait ran out (pipeline stalled)     */
+  MLA_ERR_DEVICE_OOB = 6,           /* a block-table entry or sequence index out of range     */
+  MLA_ERR_DEVICE_BAD_LENGTH = 7     /* seq_len < number of query tokens, or beyond the table  */
+} mla_status;
+
+typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1 } mla_dtype;
+
+/*
+ * Model dimensions, named as in the page's module (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」
+ * §2): n_heads, dim (d_model), kv_lora_rank (d_c), qk_rope_head_dim (d_rope),
+ * qk_nope_head_dim (d_nope), v_head_dim (d_v). softmax_scale is normally
+ * 1/sqrt(d_nope + d_rope) (the module's self.scale). rms_eps is the kv_norm epsilon.
+ * rope_theta is the RoPE base: pair i of a d_rope-wide vector at position p turns by
+ * p * rope_theta^(-2i/d_rope) (「淺析DeepSeek多頭潛在注意力機制（MLA）」, "MLA與ROPE的融合";
+ * pairs are adjacent elements (2i, 2i+1)). page_size is the number of tokens per cache page.
+ */
+typedef struct {
+  int32_t n_heads;
+  int32_t d_model;
+  int32_t d_c;
+  int32_t d_rope;
+  int32_t d_nope;
+  int32_t d_v;
+  int32_t page_size;
+  int32_t dtype; /* mla_dtype */
+  float softmax_scale;
+  float rms_eps;
+  float rope_theta;
+} mla_config;
+
+/* Human-readable name of a status code (static string). */
+const char* mla_status_string(mla_status status);
+
+/*
+ * Split the key/value up-projection into the two absorbed weight packs.
+ * Source: the module's wkv_b (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2), whose output is
+ * viewed as (n_heads, d_nope + d_v) and split into the no-rope key part and the value part.
+ *   wkv_b  [n_heads*(d_nope+d_v), d_c]   input
+ *   w_uk_t [n_heads, d_c, d_nope]        output: w_uk_t[h][c][n] = wkv_b[h*(d_nope+d_v)+n][c]
+ *                                        (W_UK[h] transposed, so q_lat = q_nope · W_UK[h])
+ *   w_uv   [n_heads, d_v, d_c]           output: w_uv[h][v][c] = wkv_b[h*(d_nope+d_v)+d_nope+v][c]
+ * A pure re-indexing copy: bit-exact. Buffers must not overlap.
+ */
+mla_status mla_absorb_weights(const mla_config* cfg, const void* wkv_b, void* w_uk_t,
+                              void* w_uv, void* stream);
+
+/* Bytes of workspace mla_append_latent needs for n_tok tokens (0 if the arguments are invalid). */
+size_t mla_append_workspace_size(const mla_config* cfg, int32_t n_tok);
+
+/*
+ * Append n_tok tokens to the paged latent cache (the KV half of the page's module, §2 of
+ * 「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」: wkv_a, split, kv_norm; plus RoPE on k_R from
+ * 「淺析DeepSeek多頭潛在注意力機制（MLA）」, "MLA與ROPE的融合"). For token i:
+ *     kv   = x[i] · w_dkvᵀ                                   (d_c + d_rope outputs)
+ *     c    = kv[:d_c] / sqrt(mean(kv[:d_c]^2) + rms_eps) * kv_gain
+ *     k_R  = RoPE(kv[d_c:], pos[i])
+ *     cache[block_table[seq_idx[i]][pos[i] / page_size]][pos[i] % page_size] = [c | k_R]
+ * rounded once to cfg->dtype. fp32 accumulation.
+ *   x           [n_tok, d_model]
+ *   w_dkv       [d_c + d_rope, d_model]     (wkv_a weight; rows [0,d_c) give c_KV)
+ *   kv_gain     [d_c]                       (kv_norm weight)
+ *   seq_idx     [n_tok] int32, in [0, batch)
+ *   pos         [n_tok] int32, 0-based position in its sequence, < max_pages*page_size
+ *   block_table [batch, max_pages] int32    page ids in [0, num_pages)
+ *   cache       [num_pages, page_size, d_c + d_rope]   updated in place, only the addressed rows
+ *   workspace   >= mla_append_workspace_size(cfg, n_tok) bytes, 256-byte aligned
+ * Tokens whose sequence, position or page is out of range are skipped and flagged
+ * MLA_ERR_DEVICE_OOB. Two tokens addressing the same row race (caller's responsibility).
+ */
+mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok,
+                             const void* w_dkv, const void* kv_gain, const int32_t* seq_idx,
+                             const int32_t* pos, const int32_t* block_table, int32_t batch,
+                             int32_t max_pages, void* cache, int32_t num_pages, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/* Bytes of workspace mla_decode needs for (batch, tq) on the current device (0 if invalid). */
+size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq);
+
+/*
+ * Batched, variable-length decode attention over the paged latent cache (absorbed form, see the
+ * top of this file), with split-KV: long sequences are cut into chunks of whole pages that run
+ * in parallel and are merged by their log-sum-exp.
+ * The cache must already hold the tq new tokens of each sequence (append first): sequence b
+ * has seq_lens[b] tokens and its query t sits at position seq_lens[b] - tq + t; it attends to
+ * tokens 0 .. seq_lens[b] - tq + t (causal among the new tokens; a query sees itself —
+ * 「淺析DeepSeek多頭潛在注意力機制（MLA）」: the new token attends to all N+1 keys).
+ *   q           [batch, tq, n_heads, d_nope + d_rope]  un-rotated queries ([q_nope | q_rope])
+ *   cache       [num_pages, page_size, d_c + d_rope]
+ *   block_table [batch, max_pages] int32
+ *   seq_lens    [batch] int32 (device), each in [tq, max_pages*page_size]
+ *   w_uk_t      [n_heads, d_c, d_nope], w_uv [n_heads, d_v, d_c]   (from mla_absorb_weights)
+ *   workspace   >= mla_decode_workspace_size(cfg, batch, tq) bytes, 256-byte aligned
+ *   out         [batch, tq, n_heads, d_v]
+ * bf16 runs on the tcgen05 tensor-core path and needs d_c = 512, d_rope = 64, d_nope = 128,
+ * d_v = 128, page_size = 64 (DeepSeek-V2 shapes); fp32 runs on CUDA cores for any shape.
+ * A sequence whose length is out of range gets zero output and MLA_ERR_DEVICE_BAD_LENGTH.
+ */
+mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                      const void* cache, int32_t num_pages, const int32_t* block_table,
+                      int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                      const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                      void* stream);
+
+/* Bytes of workspace mla_prefill_ref needs (0 if the arguments are invalid). */
+size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new);
+
+/*
+ * Reference prefill: append t_new tokens per sequence and return their attention outputs, on
+ * CUDA cores with fp32 arithmetic, for any shape and either dtype (the correctness path; the
+ * prompt pass of 「淺析DeepSeek多頭潛在注意力機制（MLA）」, "大模型的整體推理過程", done token-causal).
+ * Sequence b ends up with seq_lens[b] tokens; its new tokens take positions
+ * seq_lens[b] - t_new .. seq_lens[b] - 1 (earlier positions must already be in the cache).
+ *   x    [batch, t_new, d_model]                    hidden states of the new tokens
+ *   q    [batch, t_new, n_heads, d_nope + d_rope]   their un-rotated queries
+ *   w_dkv, kv_gain, block_table, cache: as in mla_append_latent
+ *   w_uk_t, w_uv, seq_lens: as in mla_decode (each seq_lens[b] >= t_new)
+ *   out  [batch, t_new, n_heads, d_v]
+ */
+mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, int32_t batch,
+                           int32_t t_new, const void* w_dkv, const void* kv_gain,
+                           const void* w_uk_t, const void* w_uv, const int32_t* seq_lens,
+                           const int32_t* block_table, int32_t max_pages, void* cache,
+                           int32_t num_pages, void* workspace, size_t ws_bytes, void* out,
+                           void* stream);
+
+/*
+ * Synchronise `stream`, then return (and clear) the first error a kernel of this library
+ * recorded on the current device since the previous call: MLA_OK if none. Returns
+ * MLA_ERR_CUDA if the synchronisation itself fails.
+ */
+mla_status mla_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MLA_H_ */

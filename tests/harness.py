@@ -1,0 +1,115 @@
+"""Shared helpers for the GPU parity tests: put a workload on the device, run the library,
+and build the oracle's reference from the same generator inputs (never from GPU output)."""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import torch
+
+import head_latent_attention_05_b200 as mla
+import workloads as W
+from oracle import mla_oracle as O
+
+
+def tol_bound(ref: np.ndarray, dtype: str) -> float:
+    """Parity bound: fp32 max|err| <= 1e-4 max|ref|; bf16 max|err| <= 1e-2 max|ref| + 1e-3."""
+    m = float(np.max(np.abs(ref))) if ref.size else 0.0
+    return 1e-4 * m if dtype == "f32" else 1e-2 * m + 1e-3
+
+
+def assert_parity(got, ref, dtype: str, what: str = ""):
+    got = O.f64(got)
+    ref = np.asarray(ref, dtype=np.float64)
+    assert got.shape == ref.shape, (got.shape, ref.shape)
+    assert np.all(np.isfinite(got)), f"{what}: non-finite output"
+    err = float(np.max(np.abs(got - ref))) if ref.size else 0.0
+    bound = tol_bound(ref, dtype)
+    assert err <= bound, f"{what}: max|err| {err:.3e} > bound {bound:.3e}"
+    return err, bound
+
+
+def config_of(w: W.Workload) -> mla.MlaConfig:
+    return mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, W.PAGE_SIZE, w.dtype,
+                           w.scale, w.rms_eps, w.rope_theta)
+
+
+@dataclasses.dataclass
+class Case:
+    w: W.Workload
+    cfg: mla.MlaConfig
+    lens: torch.Tensor          # host int32 [B]
+    pt: W.PageTable
+    weights: W.Weights          # host
+    cache_host: torch.Tensor    # history contents before the append (host)
+    x_new: torch.Tensor
+    seq_idx: torch.Tensor
+    pos: torch.Tensor
+    q: torch.Tensor
+    # device copies
+    d: dict
+
+
+def make_case(w: W.Workload, lens: torch.Tensor | None = None, tail_fill=None,
+              device="cuda") -> Case:
+    lens = W.seq_lens(w) if lens is None else lens.to(torch.int32)
+    pt = W.page_table(w, lens)
+    weights = W.weights(w)
+    cache = W.cache_pool(w, pt.num_pages)
+    if tail_fill is not None:
+        for page, slot in W.tail_slots(lens, pt):
+            cache[page, slot:] = tail_fill
+    x_new, seq_idx, pos, q = W.new_token_inputs(w, lens)
+    cfg = config_of(w)
+    d = dict(
+        cache=cache.to(device), block_table=pt.block_table.to(device),
+        seq_lens=lens.to(device), x_new=x_new.to(device), seq_idx=seq_idx.to(device),
+        pos=pos.to(device), q=q.contiguous().to(device), w_dkv=weights.w_dkv.to(device),
+        kv_gain=weights.kv_gain.to(device), wkv_b=weights.wkv_b.to(device),
+    )
+    dt = w.torch_dtype
+    d["w_uk_t"] = torch.empty((w.H, w.d_c, w.d_nope), dtype=dt, device=device)
+    d["w_uv"] = torch.empty((w.H, w.d_v, w.d_c), dtype=dt, device=device)
+    mla.mla_absorb_weights(cfg, d["wkv_b"], d["w_uk_t"], d["w_uv"])
+    return Case(w, cfg, lens, pt, weights, cache, x_new, seq_idx, pos, q, d)
+
+
+def run_append(c: Case):
+    ws = mla.workspace(mla.mla_append_workspace_size(c.cfg, c.x_new.shape[0]))
+    mla.mla_append_latent(c.cfg, c.d["x_new"], c.d["w_dkv"], c.d["kv_gain"], c.d["seq_idx"],
+                          c.d["pos"], c.d["block_table"], c.d["cache"], ws)
+
+
+def run_decode(c: Case) -> torch.Tensor:
+    w = c.w
+    out = torch.empty((w.B, w.Tq, w.H, w.d_v), dtype=w.torch_dtype, device="cuda")
+    ws = mla.workspace(mla.mla_decode_workspace_size(c.cfg, w.B, w.Tq))
+    mla.mla_decode(c.cfg, c.d["q"], c.d["cache"], c.d["block_table"], c.d["seq_lens"],
+                   c.d["w_uk_t"], c.d["w_uv"], ws, out)
+    return out
+
+
+def oracle_new_rows(c: Case) -> np.ndarray:
+    """fp64 cache rows of the appended tokens, from the oracle's own append."""
+    w = c.w
+    return O.latent_rows(c.x_new, c.weights.w_dkv, c.weights.kv_gain, c.pos.numpy(), w.d_c,
+                         w.rms_eps, w.rope_theta)
+
+
+def oracle_rows_of(c: Case, b: int, new_rows: np.ndarray) -> np.ndarray:
+    """All L_b rows of sequence b as the oracle sees them: generator history, then its own new
+    rows for the last Tq positions."""
+    w = c.w
+    L = int(c.lens[b])
+    rows = O.gather_rows(c.cache_host, c.pt.block_table[b].numpy(), L, W.PAGE_SIZE)
+    rows[L - w.Tq:] = new_rows[b * w.Tq:(b + 1) * w.Tq]
+    return rows
+
+
+def oracle_out(c: Case, b: int, heads, new_rows: np.ndarray) -> np.ndarray:
+    """Oracle output [Tq, len(heads), d_v] for sequence b (expanded form)."""
+    w = c.w
+    W_UK, W_UV = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
+    rows = oracle_rows_of(c, b, new_rows)
+    return O.decode_expanded(c.q[b], rows, W_UK, W_UV, w.scale, w.rope_theta, heads=heads)
