@@ -1,0 +1,460 @@
+#!/usr/bin/env python3
+"""Benchmark of one MLA decode step on B200: append the new tokens' latents, then decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A step is one pass of the whole hot path over one batch of synthetic input:
+mla_append_latent (down-projection GEMM + RMSNorm/RoPE/scatter) then mla_decode (plan, query
+absorption, latent attention, split combine, value projection), through the C ABI. The metric
+is cache-tokens x heads per second: sum_b L_b * Tq * H / step time, summed over all GPUs
+(each GPU decodes its own batch: weak scaling, no data-path collective).
+
+Timing: the K timed steps are captured once into a CUDA graph (so host launch latency stays
+out of device time) and replayed; before every step the graph writes 256 MiB to flush the
+126 MB L2, outside the step's CUDA events. Per-kernel times come from events the library
+records at its kernel boundaries. `e2e` repeats the step through the plain API from pinned
+host buffers, with the host->device copies of the step's inputs and the device->host copy of
+its output inside the timed region. rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import workloads as WL  # noqa: E402
+
+METRIC = "MLA decode cache-tokens/s (×heads) on 1 B200; % of HBM/tensor roofline"
+UNIT = "cache_tokens*heads/s"
+DEFAULT_WORKLOAD = "v2_bf16_b16_ctx4096"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+ATTN_PROFILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WL.WORKLOAD_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="budget of the oracle CPU-baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- bookkeeping
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def work_of(w: WL.Workload, lens: torch.Tensor) -> dict:
+    """Algorithmic work of one step (per GPU)."""
+    Ls = [int(v) for v in lens.tolist()]
+    tokens = sum(Ls)
+    elem = 4 if w.dtype == "f32" else 2
+    cache_bytes = tokens * w.row * elem
+    w_bytes = 2 * w.H * w.d_nope * w.d_c * elem          # W_UK + W_UV
+    attn_flops = sum(L * w.Tq for L in Ls) * w.H * 2 * (w.row + w.d_c)
+    proj_flops = 2 * (2 * w.B * w.Tq * w.H * w.d_nope * w.d_c)
+    return dict(units=sum(L * w.Tq for L in Ls) * w.H, tokens=tokens, cache_bytes=cache_bytes,
+                weight_bytes=w_bytes, attn_flops=attn_flops, proj_flops=proj_flops)
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled every 10 ms while running."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,utilization.gpu,"
+             "clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", "10"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.05)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(v):
+            try:
+                return float(v)
+            except ValueError:
+                return None
+        busy = [r for r in rows if (num(r[4]) or 0) > 0] or rows
+        sm = [num(r[1]) for r in busy if num(r[1]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in busy for i in range(4) if r[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": num(rows[0][2]), "reasons": reasons,
+                "samples": len(rows), "samples_busy": len(busy),
+                "power_w_max": max((num(r[3]) or 0.0) for r in rows)}
+
+
+def cpu_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+# ------------------------------------------------------------------ oracle (CPU baseline)
+
+def oracle_sample(w: WL.Workload, lens, pt, weights, cache_host, x_new, pos, q, seconds: float,
+                  max_units: int | None = None):
+    """Time the fp64 oracle (expanded form, as it stands) on (sequence, head) units of the
+    workload for about `seconds`; returns (rate in cache-tokens*heads/s, units, description)."""
+    from oracle import mla_oracle as O
+    W_UK, W_UV = O.split_wkv_b(weights.wkv_b, w.H, w.d_nope, w.d_v)
+    new_rows = O.latent_rows(x_new, weights.w_dkv, weights.kv_gain, pos.numpy(), w.d_c,
+                             w.rms_eps, w.rope_theta)
+    heads = [0, w.H // 2, w.H - 1, w.H // 3, (2 * w.H) // 3]
+    done_units, done_work, elapsed = 0, 0, 0.0
+    rows_cache = {}
+    i = 0
+    while elapsed < seconds and (max_units is None or done_units < max_units):
+        b = i % w.B
+        h = heads[(i // w.B) % len(heads)]
+        i += 1
+        L = int(lens[b])
+        if b not in rows_cache:
+            r = O.gather_rows(cache_host, pt.block_table[b].numpy(), L, WL.PAGE_SIZE)
+            r[L - w.Tq:] = new_rows[b * w.Tq:(b + 1) * w.Tq]
+            rows_cache = {b: r}
+        t0 = time.perf_counter()
+        O.decode_expanded(q[b], rows_cache[b], W_UK, W_UV, w.scale, w.rope_theta, heads=[h])
+        elapsed += time.perf_counter() - t0
+        done_units += 1
+        done_work += L * w.Tq
+    rate = done_work / elapsed if elapsed > 0 else 0.0
+    desc = (f"{done_units} (sequence, head) units of {w.name} through the fp64 expanded-form "
+            f"oracle ({done_work} cache-token*heads, {elapsed:.1f} s); rate scales to the full "
+            f"workload because the work per cache-token*head is uniform")
+    return rate, done_units, desc
+
+
+# ------------------------------------------------------------------------------- setup
+
+def build_inputs(w: WL.Workload, device):
+    lens = WL.seq_lens(w)
+    pt = WL.page_table(w, lens)
+    weights = WL.weights(w)
+    cache_host = WL.cache_pool(w, pt.num_pages)
+    x_new, seq_idx, pos, q = WL.new_token_inputs(w, lens)
+    return lens, pt, weights, cache_host, x_new, seq_idx, pos, q
+
+
+def run_reference(args, rank: int, world: int):
+    """Reference arm: the fp64 oracle on this host's cores, same workload / metric / unit."""
+    if rank != 0:
+        return
+    w = WL.WORKLOADS[args.workload]
+    lens, pt, weights, cache_host, x_new, seq_idx, pos, q = build_inputs(w, "cpu")
+    # each step: one (sequence, head) unit; the metric is total work / total time
+    for _ in range(max(0, args.warmup)):
+        oracle_sample(w, lens, pt, weights, cache_host, x_new, pos, q, 0.0, max_units=1)
+    t0 = time.perf_counter()
+    rate, units, desc = oracle_sample(w, lens, pt, weights, cache_host, x_new, pos, q,
+                                      float("inf"), max_units=args.steps)
+    wall = time.perf_counter() - t0
+    cores = cpu_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": rate, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * wall / max(1, units),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.B, "heads": w.H, "tq": w.Tq,
+                   "context": list(w.lens)},
+        "cpu_baseline": {"value": rate, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": rate, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import head_latent_attention_05_b200 as mla
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WL.WORKLOADS[args.workload]
+    lens, pt, weights, cache_host, x_new_h, seq_idx_h, pos_h, q_h = build_inputs(w, dev)
+    cfg = mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, WL.PAGE_SIZE, w.dtype,
+                          w.scale, w.rms_eps, w.rope_theta)
+    dt = w.torch_dtype
+    cache = cache_host.to(dev)
+    bt = pt.block_table.to(dev)
+    seq_lens = lens.to(dev)
+    x_new, seq_idx, pos, q = (t.contiguous().to(dev) for t in (x_new_h, seq_idx_h, pos_h, q_h))
+    w_dkv, kv_gain = weights.w_dkv.to(dev), weights.kv_gain.to(dev)
+    w_uk_t = torch.empty((w.H, w.d_c, w.d_nope), dtype=dt, device=dev)
+    w_uv = torch.empty((w.H, w.d_v, w.d_c), dtype=dt, device=dev)
+    mla.mla_absorb_weights(cfg, weights.wkv_b.to(dev), w_uk_t, w_uv)
+    n_tok = w.B * w.Tq
+    ws_a = mla.workspace(mla.mla_append_workspace_size(cfg, n_tok), dev)
+    ws_d = mla.workspace(mla.mla_decode_workspace_size(cfg, w.B, w.Tq), dev)
+    out = torch.empty((w.B, w.Tq, w.H, w.d_v), dtype=dt, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    work = work_of(w, lens)
+
+    K, Wm = args.steps, max(3, args.warmup)
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
+    step_ev = [[ev() for _ in range(8)] for _ in range(K)]   # start, 6 decode marks, end
+    # torch creates events lazily: record every event once so it exists before capture
+    for evs in step_ev:
+        for e in evs:
+            e.record()
+    torch.cuda.synchronize()
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record()
+        mla.mla_append_latent(cfg, x_new, w_dkv, kv_gain, seq_idx, pos, bt, cache, ws_a)
+        if evs is not None:
+            mla.mla_decode_profiled(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out,
+                                    evs[1:7])
+            evs[7].record()
+        else:
+            mla.mla_decode(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out)
+
+    # warm-up (eager), then a correctness guard: no device error may be pending
+    for i in range(Wm):
+        flush.fill_(i & 0xFF)
+        step()
+    err = mla.mla_get_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error during warm-up: {mla.mla_status_string(err)}")
+
+    graph = None
+    if not args.no_graph:
+        graph = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream(device=dev)
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(graph, stream=s):
+                for i in range(K):
+                    flush.fill_((i * 7) & 0xFF)
+                    step(step_ev[i])
+        torch.cuda.current_stream().wait_stream(s)
+        torch.cuda.synchronize()
+
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.03)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.perf_counter()
+    if graph is not None:
+        graph.replay()
+    else:
+        for i in range(K):
+            flush.fill_((i * 7) & 0xFF)
+            step(step_ev[i])
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    if world > 1:
+        torch.distributed.barrier()
+    clk = clocks.stop()
+    err = mla.mla_get_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error in the timed region: {mla.mla_status_string(err)}")
+
+    names = ["append", "plan", "q_absorb", "attention", "combine", "value_proj"]
+    per = {n: [] for n in names}
+    steps_ms = []
+    for evs in step_ev:
+        steps_ms.append(evs[0].elapsed_time(evs[7]))
+        for j, n in enumerate(names):
+            per[n].append(evs[j].elapsed_time(evs[j + 1]))
+    total_ms = sum(steps_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / K
+    value = world * work["units"] / (ms_per_step / 1e3)
+    kernel_ms = {n: statistics.fmean(v) for n, v in per.items()}
+
+    # ---- e2e through the plain API from pinned host buffers
+    x_pin = x_new_h.contiguous().pin_memory()
+    q_pin = q_h.contiguous().pin_memory()
+    sl_pin, si_pin, pos_pin = (t.contiguous().pin_memory() for t in (lens, seq_idx_h, pos_h))
+    out_pin = torch.empty(out.shape, dtype=dt).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (x_pin, q_pin, sl_pin, si_pin, pos_pin))
+    d2h = out_pin.numel() * out_pin.element_size()
+    K2 = min(K, 50)
+    e2e_ev = [(ev(), ev()) for _ in range(K2)]
+    e2e_ms = []
+    for i in range(K2):
+        flush.fill_(i & 0xFF)
+        a, b = e2e_ev[i]
+        a.record()
+        x_new.copy_(x_pin, non_blocking=True)
+        q.copy_(q_pin, non_blocking=True)
+        seq_lens.copy_(sl_pin, non_blocking=True)
+        seq_idx.copy_(si_pin, non_blocking=True)
+        pos.copy_(pos_pin, non_blocking=True)
+        step()
+        out_pin.copy_(out, non_blocking=True)
+        b.record()
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    e2e_step = statistics.fmean(e2e_ms)
+    if world > 1:
+        t = torch.tensor([e2e_step], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_step = float(t.item())
+    err = mla.mla_get_device_error()
+    if err != 0:
+        raise RuntimeError(f"device error in the e2e loop: {mla.mla_status_string(err)}")
+
+    # ---- roofline of the dominant kernel (latent attention)
+    pk, pk_kind = peaks()
+    t_attn = kernel_ms["attention"] / 1e3
+    hbm_peak = float(pk["hbm_gbs"])
+    tc_peak = float(pk["bf16_tflops"])
+    t_mem = work["cache_bytes"] / (hbm_peak * 1e9)
+    t_tc = work["attn_flops"] / (tc_peak * 1e12)
+    bound = "hbm" if t_mem >= t_tc else "tensor"
+    traffic = None
+    if os.path.exists(ATTN_PROFILE):
+        with open(ATTN_PROFILE) as f:
+            prof = json.load(f)
+        if prof.get("workload") == w.name and prof.get("kernel_source_sha") == kernel_sha():
+            traffic = prof.get("dram_bytes_per_launch")
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": work["cache_bytes"] / t_attn / 1e9, "peak": hbm_peak,
+                "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": work["attn_flops"] / t_attn / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = traffic
+    roof["peak_source"] = f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback"
+    roof["kernel"] = "mla_decode_attn_kernel"
+    roof["algorithmic_bytes_per_launch"] = work["cache_bytes"]
+    roof["algorithmic_flops_per_launch"] = work["attn_flops"]
+    roof["tensor_achieved_tflops"] = work["attn_flops"] / t_attn / 1e12
+    roof["step_roofline_frac"] = max(
+        (work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
+        (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12)) / (ms_per_step / 1e3)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": {"workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
+                   "heads": w.H, "tq": w.Tq, "context": list(w.lens),
+                   "cache_tokens_per_gpu": work["tokens"], "parallelism": f"dp{world}",
+                   "l2": "flushed before every step (256 MiB write, outside the step events)",
+                   "timing": "CUDA graph of the K steps" if graph is not None else "eager",
+                   "step": "mla_append_latent + mla_decode"},
+        "roofline": roof,
+        "kernel_ms": kernel_ms,
+        "e2e": {"value": world * work["units"] / (e2e_step / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step},
+        "gpu_launches": K * 7,
+        "clocks": clk,
+        "wall_s_timed_region": t_wall,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, units, desc = oracle_sample(w, lens, pt, weights, cache_host, x_new_h, pos_h, q_h,
+                                          args.cpu_seconds)
+        line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cpu_threads(),
+                                "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    del graph
+
+
+def kernel_sha() -> str:
+    """Hash of the attention kernel source, to tell whether stored counters are current."""
+    import hashlib
+    path = os.path.join(ROOT, "head_latent_attention_05_b200", "csrc", "tc_decode.cuh")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def main():
+    args = parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (the library has no CPU path)")
+    from head_latent_attention_05_b200 import build as _b
+    if rank == 0 or world == 1:
+        _b.build()
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group(
+            "nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local_rank))
+        torch.distributed.barrier()
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -29,7 +29,8 @@ STATUS = {
 # Every symbol include/mla.h declares (checked by the tests against the built library).
 EXPORTED = (
     "mla_status_string", "mla_absorb_weights", "mla_append_workspace_size", "mla_append_latent",
-    "mla_decode_workspace_size", "mla_decode", "mla_prefill_ref_workspace_size",
+    "mla_decode_workspace_size", "mla_decode", "mla_decode_profiled",
+    "mla_prefill_ref_workspace_size",
     "mla_prefill_ref", "mla_get_device_error",
 )
 
@@ -80,6 +81,8 @@ def load_library() -> ctypes.CDLL:
         "mla_append_latent": (ctypes.c_int, [CFG, P, I32, P, P, P, P, P, I32, I32, P, I32, P, SZ, P]),
         "mla_decode_workspace_size": (SZ, [CFG, I32, I32]),
         "mla_decode": (ctypes.c_int, [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P, P]),
+        "mla_decode_profiled": (ctypes.c_int,
+                                [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P, P, P]),
         "mla_prefill_ref_workspace_size": (SZ, [CFG, I32, I32]),
         "mla_prefill_ref": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ, P, P]),
         "mla_get_device_error": (ctypes.c_int, [P]),
@@ -142,6 +145,23 @@ def mla_decode(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv, wo
         ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),
         block_table.shape[1], _ptr(seq_lens), _ptr(w_uk_t), _ptr(w_uv), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)), "mla_decode")
+
+
+def mla_decode_profiled(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv,
+                        workspace, out, events, stream=None):
+    """mla_decode that also records 6 torch.cuda.Event objects at its kernel boundaries.
+
+    The events must already exist on the device (torch creates them lazily: record each once
+    before the first call). Create them with external=True to time inside a CUDA graph."""
+    if len(events) != 6 or any(e.cuda_event == 0 for e in events):
+        raise ValueError("mla_decode_profiled needs 6 already-created CUDA events")
+    arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    batch, tq = q.shape[0], q.shape[1]
+    _check(load_library().mla_decode_profiled(
+        ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), _ptr(w_uk_t), _ptr(w_uv), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream), arr),
+        "mla_decode_profiled")
 
 
 def mla_prefill_ref_workspace_size(cfg: MlaConfig, batch: int, t_new: int) -> int:

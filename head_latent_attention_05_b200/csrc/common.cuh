@@ -80,16 +80,18 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 }
 
 // RoPE of one pair (x, y) = (v[2i], v[2i+1]) at position pos: turn by pos * theta^(-2i/d).
-// The angle is formed and reduced in double precision so that positions up to 2^17 keep
-// full fp32 accuracy in the result.
+// The angle is formed in double precision and reduced to [-pi, pi] there, so that positions
+// up to 2^17 keep full fp32 accuracy; the rotation itself is done in fp32.
 __device__ __forceinline__ void rope_pair(float x, float y, int pair, int d, int pos,
                                           float theta, float* ox, float* oy) {
-  const double inv_freq = pow(static_cast<double>(theta), -2.0 * pair / static_cast<double>(d));
-  double s, c;
-  sincos(static_cast<double>(pos) * inv_freq, &s, &c);
-  const double xd = x, yd = y;
-  *ox = static_cast<float>(xd * c - yd * s);
-  *oy = static_cast<float>(xd * s + yd * c);
+  const double two_pi = 6.283185307179586476925286766559;
+  const double inv_freq = exp2(-(2.0 * pair / static_cast<double>(d)) * log2(static_cast<double>(theta)));
+  const double ang = static_cast<double>(pos) * inv_freq;
+  const float r = static_cast<float>(ang - two_pi * rint(ang / two_pi));
+  float s, c;
+  sincosf(r, &s, &c);
+  *ox = x * c - y * s;
+  *oy = x * s + y * c;
 }
 
 }  // namespace mla

@@ -10,6 +10,7 @@
 #include <cstdint>
 #include <cstring>
 #include <mutex>
+#include <unordered_map>
 
 #include "../../include/mla.h"
 #include "common.cuh"
@@ -112,12 +113,35 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Largest dynamic shared memory a kernel asks for: raise its limit once per device.
+// Raise a kernel's dynamic shared-memory limit, once per (kernel, device): later calls, which
+// may be inside a CUDA-graph capture, then make no CUDA runtime call here at all.
 template <typename K>
 bool allow_smem(K kernel, int bytes) {
   if (bytes <= 48 * 1024) return true;
-  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) ==
-         cudaSuccess;
+  static std::mutex mu;
+  static std::unordered_map<const void*, uint64_t> done;  // kernel -> bitmask of devices
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev >= 64) return false;
+  const void* key = reinterpret_cast<const void*>(kernel);
+  std::lock_guard<std::mutex> lock(mu);
+  uint64_t& mask = done[key];
+  if (mask & (1ull << dev)) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) !=
+      cudaSuccess)
+    return false;
+  mask |= 1ull << dev;
+  return true;
+}
+
+// Record a profiling event: as an event-record node of the graph while the stream is being
+// captured, as a plain record otherwise.
+void record_mark(cudaEvent_t ev, cudaStream_t st) {
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  cudaStreamIsCapturing(st, &cs);
+  if (cs == cudaStreamCaptureStatusActive)
+    cudaEventRecordWithFlags(ev, st, cudaEventRecordExternal);
+  else
+    cudaEventRecord(ev, st);
 }
 
 // ------------------------------------------------------------------ tcgen05 GEMM launcher
@@ -164,11 +188,17 @@ AppendPlan append_plan(const mla_config* c, int n_tok) {
   p.k_chunks = c->d_model / 64;
   const int n_tiles = (n_tok + 255) / 256;
   const int sms = device_sm_count() > 0 ? device_sm_count() : 148;
-  int splits = (2 * sms + p.m_tiles * n_tiles - 1) / (p.m_tiles * n_tiles);
+  int splits = (sms + p.m_tiles * n_tiles - 1) / (p.m_tiles * n_tiles);
   splits = splits < 1 ? 1 : (splits > p.k_chunks ? p.k_chunks : splits);
   p.chunks_per_split = (p.k_chunks + splits - 1) / splits;
   p.k_splits = (p.k_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
   return p;
+}
+
+// One thread per cache-row feature (a multiple of 32, at most 1024).
+int finish_threads(int row) {
+  const int t = (row + 31) / 32 * 32;
+  return t > 1024 ? 1024 : t;
 }
 
 bool tc_append_shape(const mla_config* c) {
@@ -186,10 +216,16 @@ struct DecodeLayout {
   size_t bytes;
 };
 
+// Number of CTA pairs of the attention kernel: one CTA per SM (its shared memory and TMEM fill
+// an SM), two CTAs per pair.
+int attn_pairs() {
+  const int sms = device_sm_count();
+  return (sms >= 2 ? sms : 2) / 2;
+}
+
 DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
   DecodeLayout L{};
-  const int sms = device_sm_count();
-  L.P = (sms >= 2 ? sms : 2) / 2;
+  L.P = attn_pairs();
   L.R = Tq * c->n_heads;
   L.n_mt = (L.R + 127) / 128;
   L.U = B * L.n_mt;
@@ -231,7 +267,12 @@ template <typename T>
 mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const void* cache,
                        int num_pages, const int32_t* block_table, int max_pages,
                        const int32_t* seq_lens, const void* w_uk_t, const void* w_uv,
-                       const SimtLayout& L, void* out, cudaStream_t st) {
+                       const SimtLayout& L, void* out, cudaStream_t st,
+                       void* const* events = nullptr) {
+  auto mark = [&](int i) {
+    if (events != nullptr && events[i] != nullptr)
+      record_mark(static_cast<cudaEvent_t>(events[i]), st);
+  };
   const int rows = B * Tq * c->n_heads;
   const int row = c->d_c + c->d_rope;
   const int max_pos = max_pages * c->page_size;
@@ -240,9 +281,12 @@ mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const 
       Tq, c->d_c, c->d_rope, c->d_nope, max_pos, c->rope_theta);
   const int attn_smem = (row + c->d_c) * static_cast<int>(sizeof(float));
   if (!allow_smem(attn_simt_kernel<T>, attn_smem)) return MLA_ERR_CUDA;
+  mark(2);
   attn_simt_kernel<T><<<rows, 256, attn_smem, st>>>(
       L.qhat, static_cast<const T*>(cache), block_table, seq_lens, L.o_lat, c->n_heads, Tq,
       c->d_c, c->d_rope, max_pages, num_pages, c->page_size, c->softmax_scale);
+  mark(3);
+  mark(4);
   outproj_simt_kernel<T><<<rows, 256, c->d_c * sizeof(float), st>>>(
       L.o_lat, static_cast<const T*>(w_uv), static_cast<T*>(out), c->n_heads, c->d_c, c->d_v);
   return last_launch_status();
@@ -258,7 +302,7 @@ mla_status simt_append(const mla_config* c, const void* x, int n_tok, const void
   linear_rows_kernel<T><<<g1, 256, 0, st>>>(static_cast<const T*>(x),
                                             static_cast<const T*>(w_dkv), kv, n_tok, row,
                                             c->d_model);
-  append_finish_kernel<T><<<n_tok, 256, row * sizeof(float), st>>>(
+  append_finish_kernel<T><<<n_tok, finish_threads(row), row * sizeof(float), st>>>(
       kv, 1, n_tok, static_cast<const T*>(kv_gain), seq_idx, pos, block_table, batch,
       max_pages, static_cast<T*>(cache), num_pages, c->page_size, c->d_c, c->d_rope,
       c->rms_eps, c->rope_theta);
@@ -368,7 +412,7 @@ mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok
   EpiSplitK epi{partial, n_tok, row};
   mla_status s = launch_gemm(mA, mB, shp, ap.m_tiles, 1, epi, st);
   if (s != MLA_OK) return s;
-  append_finish_kernel<__nv_bfloat16><<<n_tok, 256, row * sizeof(float), st>>>(
+  append_finish_kernel<__nv_bfloat16><<<n_tok, finish_threads(row), row * sizeof(float), st>>>(
       partial, ap.k_splits, n_tok, static_cast<const __nv_bfloat16*>(kv_gain), seq_idx, pos,
       block_table, batch, max_pages, static_cast<__nv_bfloat16*>(cache), num_pages,
       cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps, cfg->rope_theta);
@@ -384,11 +428,11 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t t
   return simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, nullptr).bytes;
 }
 
-mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
-                      const void* cache, int32_t num_pages, const int32_t* block_table,
-                      int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
-                      const void* w_uv, void* workspace, size_t ws_bytes, void* out,
-                      void* stream) {
+static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                              const void* cache, int32_t num_pages, const int32_t* block_table,
+                              int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                              const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                              void* stream, void* const* events) {
   const mla_status cs = check_config(cfg);
   if (cs != MLA_OK) return cs;
   if (batch < 1 || tq < 1 || num_pages < 1 || max_pages < 1) return MLA_ERR_INVALID_ARG;
@@ -399,11 +443,22 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
   if (cfg->dtype == MLA_DTYPE_BF16 && !tc_decode_shape(cfg)) return MLA_ERR_UNSUPPORTED;
   if (ws_bytes < mla_decode_workspace_size(cfg, batch, tq)) return MLA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // events[i] (if given) is recorded before kernel i: plan, q absorption, attention, combine,
+  // value projection; events[5] after the last one.
+  auto mark = [&](int i) {
+    if (events != nullptr && events[i] != nullptr)
+      record_mark(static_cast<cudaEvent_t>(events[i]), st);
+  };
 
   if (cfg->dtype == MLA_DTYPE_F32) {
     const SimtLayout L = simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, workspace);
-    return simt_decode<float>(cfg, q, batch, tq, cache, num_pages, block_table, max_pages,
-                              seq_lens, w_uk_t, w_uv, L, out, st);
+    mark(0);
+    mark(1);
+    const mla_status s = simt_decode<float>(cfg, q, batch, tq, cache, num_pages, block_table,
+                                            max_pages, seq_lens, w_uk_t, w_uv, L, out, st,
+                                            events);
+    mark(5);
+    return s;
   }
 
   const DecodeLayout L = decode_layout_tc(cfg, batch, tq, workspace);
@@ -413,11 +468,13 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
   const int qrow = cfg->d_nope + cfg->d_rope;
 
   // (1) plan the split-KV work list on the device
+  mark(0);
   PlanParams pp{seq_lens, batch, tq, L.n_mt, max_pos, L.P, L.max_segs,
                 L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
   attn_plan_kernel<<<1, 1024, 0, st>>>(pp);
 
   // (2) Q̂ = [q_nope · W_UK | RoPE(q_rope)]
+  mark(1);
   {
     CUtensorMap mA, mB;
     const uint64_t da[3] = {static_cast<uint64_t>(cfg->d_nope), ATT_DC, static_cast<uint64_t>(H)};
@@ -447,16 +504,19 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
     const uint32_t bq[2] = {64, 128};
     if (!make_map(&mc, cache, 2, dc, sc, bc) || !make_map(&mq, L.qhat, 2, dq, sc, bq))
       return MLA_ERR_CUDA;
-    AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
+    AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat,
+                  static_cast<const __nv_bfloat16*>(cache), L.o_part, L.lse,
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
                   cfg->softmax_scale * 1.4426950408889634f};
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
+    mark(2);
     mla_decode_attn_kernel<<<2 * L.P, ATT_THREADS, ATT_SMEM_BYTES, st>>>(mc, mq, ap);
     const mla_status s = last_launch_status();
     if (s != MLA_OK) return s;
   }
 
   // (4) merge split partials -> o_lat (bf16)
+  mark(3);
   {
     const int rows = batch * L.R;
     attn_combine_kernel<<<(rows + 7) / 8, 256, 0, st>>>(L.o_part, L.lse, L.unit_seg, L.o_lat,
@@ -478,8 +538,30 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
       return MLA_ERR_CUDA;
     GemmShape shp{cfg->d_v, n_q, ATT_DC / 64, ATT_DC / 64, 1, 1};
     EpiOut epi{static_cast<__nv_bfloat16*>(out), H, cfg->d_v};
-    return launch_gemm(mA, mB, shp, (cfg->d_v + 127) / 128, H, epi, st);
+    mark(4);
+    const mla_status s = launch_gemm(mA, mB, shp, (cfg->d_v + 127) / 128, H, epi, st);
+    mark(5);
+    return s;
   }
+}
+
+mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                      const void* cache, int32_t num_pages, const int32_t* block_table,
+                      int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                      const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                      void* stream) {
+  return decode_impl(cfg, q, batch, tq, cache, num_pages, block_table, max_pages, seq_lens,
+                     w_uk_t, w_uv, workspace, ws_bytes, out, stream, nullptr);
+}
+
+mla_status mla_decode_profiled(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                               const void* cache, int32_t num_pages, const int32_t* block_table,
+                               int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                               const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                               void* stream, void* const* events) {
+  if (events == nullptr) return MLA_ERR_INVALID_ARG;
+  return decode_impl(cfg, q, batch, tq, cache, num_pages, block_table, max_pages, seq_lens,
+                     w_uk_t, w_uv, workspace, ws_bytes, out, stream, events);
 }
 
 size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new) {

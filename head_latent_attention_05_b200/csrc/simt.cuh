@@ -67,9 +67,10 @@ __device__ __forceinline__ T* cache_row(T* cache, const int32_t* block_table, in
 
 // Per token: RMSNorm over c_KV, RoPE on k_R at the token's position, one rounding to the
 // cache type, scatter to its page slot. kv holds n_splits partial sums [n_splits][n_tok][row],
-// added in a fixed order.
+// added in a fixed order. One thread per feature (blockDim >= row), so the partial sums of a
+// row are read in parallel.
 template <typename T>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(1024)
 append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
                      const T* __restrict__ kv_gain, const int32_t* __restrict__ seq_idx,
                      const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table,
@@ -87,8 +88,11 @@ append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
   }
   float ss = 0.0f;
   for (int f = threadIdx.x; f < row; f += blockDim.x) {
+    const float* src = kv + static_cast<int64_t>(i) * row + f;
+    const int64_t stride = static_cast<int64_t>(n_tok) * row;
     float v = 0.0f;
-    for (int s = 0; s < n_splits; ++s) v += kv[(static_cast<int64_t>(s) * n_tok + i) * row + f];
+#pragma unroll 8
+    for (int s = 0; s < n_splits; ++s) v += src[s * stride];
     row_s[f] = v;
     if (f < d_c) ss = fmaf(v, v, ss);
   }

@@ -8,20 +8,33 @@
 // the combine kernel merges by log-sum-exp.
 //
 // One pair of CTAs per range. Both CTAs run the same token tiles: each computes the full
-// score tile S = Q̂·Cᵀ (K = 576) and the same softmax, and accumulates its own half of the
-// latent output O[:, half*256 : half*256+256] += P·C[:, half]. Splitting d_c this way keeps
-// the fp32 accumulator within TMEM (256 columns per CTA) without any cross-CTA exchange.
+// score tile S = Q̂·Cᵀ (K = 576, heads on the MMA M side) and the same softmax, and accumulates
+// its own half of the latent output O[:, half*256 : half*256+256] += P·C[:, half]. Splitting
+// d_c keeps the fp32 accumulator within TMEM (256 columns per CTA). The pair shares nothing:
+// exchanging partial scores through distributed shared memory instead of recomputing them
+// measured slower on B200 (DSMEM moves ~8 bytes/clock per SM).
 //
 // Per CTA: TMEM columns [0,256) O half, [256,320) S, [320,512) Q̂[:, 0:384] as bf16 pairs (the
 // A operand of the first 24 K-steps of S). Shared memory: 2 stages x 9 chunks of
 // [64 tokens x 64 dims] (the whole 576-wide page, 128-byte swizzle, one TMA box per chunk),
 // Q̂[:, 384:576] (3 chunks of [128 x 64]) and P [128 x 64] bf16.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA issuer, warps 2..5
-// softmax / rescale / epilogue (warp w owns TMEM lanes 32*(w%4).., i.e. query rows).
+// Each stage is released in two parts: the 5 chunks only the score MMA reads (the other half's
+// c_KV and k_R) as soon as S is computed, the 4 chunks of this CTA's c_KV half after P·C. The
+// score MMA consumes the early chunks first, so the late chunks' load latency hides behind it.
+//
+// Warp roles (352 threads): warp 0 TMA producer, warp 1 issues the score MMAs, warp 6 issues
+// the P·C MMAs (a single thread issues at most one tcgen05.mma per ~48 cycles, so the two
+// streams get their own threads; each accumulator still has a single issuer, which keeps the
+// summation order, and the result, deterministic). Warps 2..5 and 7..10 run the softmax,
+// rescale and epilogue: warp w owns TMEM lanes 32*(w%4).. (query rows), and the two warps of a
+// lane quarter split each row's 64 scores (columns 0..31 and 32..63), agreeing on the row
+// maximum through shared memory once per tile.
 // Online softmax in base 2 with a lazy rescale: the running maximum only moves (and O is
 // rescaled) when a new score exceeds it by more than 2^8, which keeps every P <= 256.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 #include "ptx.cuh"
@@ -40,11 +53,13 @@ constexpr int ATT_QT_ELEMS = 384;                 // Q̂ columns kept in TMEM
 constexpr int ATT_QS_CHUNKS = (ATT_ROW - ATT_QT_ELEMS) / 64;   // 3 chunks of Q̂ in smem
 constexpr int ATT_QS_CHUNK_BYTES = 128 * 128;     // [128 rows x 64 bf16]
 constexpr int ATT_P_BYTES = 128 * 128;            // P [128 x 64] bf16
-constexpr int ATT_THREADS = 192;
+constexpr int ATT_THREADS = 352;
+constexpr int ATT_SM_WARPS = 8;                   // softmax warps: 2 per TMEM lane quarter
 constexpr int ATT_SMEM_BYTES =
     ATT_STAGES * ATT_TILE_BYTES + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES + ATT_P_BYTES + 1024;
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;     // log2 units
+constexpr int ATT_PREFETCH_AHEAD = 4;             // pages prefetched into L2 ahead of the loads
 
 struct AttnSeg {
   int32_t unit;        // b * n_mt + mt
@@ -59,6 +74,7 @@ struct AttnParams {
   const AttnSeg* segs;
   const int32_t* pair_seg;   // [P + 1]: pair p runs segments [pair_seg[p], pair_seg[p+1])
   const __nv_bfloat16* qhat; // [B*R][576]
+  const __nv_bfloat16* cache;  // [num_pages][64][576] (for L2 prefetch)
   float* o_part;             // [max_segs][128][512]
   float* lse;                // [max_segs][128]   (base-2 log-sum-exp of the scaled scores)
   int max_pages, num_pages;
@@ -144,35 +160,40 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
   }
   const int64_t T = carry_s;
   __syncthreads();
-  // pass 2: segments per unit (one per pair its tile range touches)
+  // pass 2: segments per unit: one per pair whose (non-empty) tile range meets the unit's.
+  // When there are fewer tiles than pairs some pair ranges are empty; they get no segment.
   if (threadIdx.x == 0) carry_s = 0;
   __syncthreads();
   for (int u0 = 0; u0 < U; u0 += 1024) {
     const int u = u0 + threadIdx.x;
-    int nseg = 0, t0 = 0, t1 = 0;
+    int nseg = 0, t0 = 0, t1 = 0, p0 = 0, p1 = -1;
     if (u < U) {
       t0 = pp.unit_tiles[u];
       t1 = (u + 1 < U) ? pp.unit_tiles[u + 1] : static_cast<int>(T);
-      if (t1 > t0) nseg = pair_of(t1 - 1, T, pp.P) - pair_of(t0, T, pp.P) + 1;
+      if (t1 > t0) {
+        p0 = pair_of(t0, T, pp.P);
+        p1 = pair_of(t1 - 1, T, pp.P);
+        for (int p = p0; p <= p1; ++p)
+          nseg += pair_start(p, T, pp.P) < pair_start(p + 1, T, pp.P) ? 1 : 0;
+      }
     }
     int excl;
     const int tot = block_exclusive_scan(nseg, &excl, warp_tot);
     if (u < U) {
       const int s0 = carry_s + excl;
       pp.unit_seg[u] = s0;
-      if (nseg > 0) {
-        const int p0 = pair_of(t0, T, pp.P);
-        for (int i = 0; i < nseg; ++i) {
-          const int p = p0 + i;
-          const int64_t a = max(static_cast<int64_t>(t0), pair_start(p, T, pp.P));
-          const int64_t e = min(static_cast<int64_t>(t1), pair_start(p + 1, T, pp.P));
-          AttnSeg sg;
-          sg.unit = u;
-          sg.tile_begin = static_cast<int32_t>(a - t0);
-          sg.tile_end = static_cast<int32_t>(e - t0);
-          sg.pair = p;
-          if (s0 + i < pp.max_segs) pp.segs[s0 + i] = sg;
-        }
+      int i = 0;
+      for (int p = p0; p <= p1; ++p) {
+        const int64_t a = max(static_cast<int64_t>(t0), pair_start(p, T, pp.P));
+        const int64_t e = min(static_cast<int64_t>(t1), pair_start(p + 1, T, pp.P));
+        if (e <= a) continue;
+        AttnSeg sg;
+        sg.unit = u;
+        sg.tile_begin = static_cast<int32_t>(a - t0);
+        sg.tile_end = static_cast<int32_t>(e - t0);
+        sg.pair = p;
+        if (s0 + i < pp.max_segs) pp.segs[s0 + i] = sg;
+        ++i;
       }
     }
     __syncthreads();
@@ -197,9 +218,12 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
 // ------------------------------------------------------------------------ attention kernel
 
 struct AttnShared {
-  uint64_t tile_full[ATT_STAGES];
-  uint64_t tile_empty[ATT_STAGES];
+  uint64_t full_qk[ATT_STAGES], full_own[ATT_STAGES];    // stage chunks landed (TMA)
+  uint64_t empty_qk[ATT_STAGES], empty_own[ATT_STAGES];  // stage chunks free again (MMA commit)
   uint64_t q_full, q_free, s_full, s_free, p_full, pv_done, o_free, drain;
+  uint64_t pair_bar[4];            // the two softmax warps of a lane quarter meet here
+  float row_max[2][2][128];        // [tile parity][column half][row] partial row maxima
+  float row_sum[2][128];           // [column half][row] partial row sums of a segment
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -228,13 +252,59 @@ __device__ __forceinline__ bool att_warp_wait(AttnShared& sh, uint64_t* bar, uin
   return ok;
 }
 
+// Walks the tiles of a CTA's segments in order: (segment index, tile within the unit).
+struct TileCursor {
+  const AttnSeg* segs;
+  int s_i, s_end, tile, k;   // k: segment counter (0-based) within the CTA
+  AttnSeg sg;
+  __device__ void init(const AttnSeg* sg_ptr, int begin, int end) {
+    segs = sg_ptr; s_i = begin; s_end = end; k = 0;
+    if (s_i < s_end) { sg = segs[s_i]; tile = sg.tile_begin; }
+  }
+  __device__ bool valid() const { return s_i < s_end; }
+  __device__ bool first_of_seg() const { return tile == sg.tile_begin; }
+  __device__ bool last_of_seg() const { return tile + 1 == sg.tile_end; }
+  __device__ void next() {
+    if (++tile >= sg.tile_end) {
+      ++s_i; ++k;
+      if (s_i < s_end) { sg = segs[s_i]; tile = sg.tile_begin; }
+    }
+  }
+};
+
+// Chunk j of a tile in the order the score MMA consumes it: first the 5 chunks only it needs
+// (the other half's 4 c_KV chunks, then k_R), then this CTA's own 4 c_KV chunks.
+__device__ __forceinline__ int att_chunk_order(int half, int j) {
+  return j < 4 ? 4 * (1 - half) + j : (j == 4 ? 8 : 4 * half + (j - 5));
+}
+
+// Four K = 16 steps of S over chunk C = att_chunk_order(HALF, J) of a stage: A = Q̂[:, 64C ..
+// 64C+63] (TMEM for C < 6, the smem part above), B = the stage's chunk C. J == 0 overwrites S.
+template <int HALF, int J>
+__device__ __forceinline__ void att_qk_chunk(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc) {
+  constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
+  constexpr int C = J < 4 ? 4 * (1 - HALF) + J : (J == 4 ? 8 : 4 * HALF + (J - 5));
+  const uint64_t b0 = b_stage + static_cast<uint64_t>((C * ATT_CHUNK_BYTES) >> 4);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    const uint32_t acc = (J == 0 && kk == 0) ? 0u : 1u;
+    if constexpr (C < ATT_QT_ELEMS / 64)
+      mma_bf16_ts(tmem + TM_S, tmem + TM_Q + (C * 4 + kk) * 8, b0 + static_cast<uint64_t>(kk * 2),
+                  IDESC_QK, acc);
+    else
+      mma_bf16_ss(tmem + TM_S,
+                  qs_desc + static_cast<uint64_t>(((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES + kk * 32) >> 4),
+                  b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
+  }
+}
+
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                        const __grid_constant__ CUtensorMap map_qhat, AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* stage_buf = smem;
+  uint8_t* stage_buf = smem;   // chunk c of stage s at stage_buf + s*TILE + c*CHUNK
   uint8_t* qs_buf = smem + ATT_STAGES * ATT_TILE_BYTES;
   uint8_t* p_buf = qs_buf + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES;
   __shared__ AttnShared sh;
@@ -245,17 +315,20 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ATT_STAGES; ++s) {
-      mbar_init(&sh.tile_full[s], 1);
-      mbar_init(&sh.tile_empty[s], 1);
+      mbar_init(&sh.full_qk[s], 1);
+      mbar_init(&sh.full_own[s], 1);
+      mbar_init(&sh.empty_qk[s], 1);
+      mbar_init(&sh.empty_own[s], 2);   // both MMA threads read a stage's own chunks
     }
-    mbar_init(&sh.q_full, 1 + 4);
+    mbar_init(&sh.q_full, 1 + ATT_SM_WARPS);
     mbar_init(&sh.q_free, 1);
     mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.s_free, 4);
-    mbar_init(&sh.p_full, 4);
+    mbar_init(&sh.s_free, ATT_SM_WARPS);
+    mbar_init(&sh.p_full, ATT_SM_WARPS);
     mbar_init(&sh.pv_done, 1);
-    mbar_init(&sh.o_free, 4);
-    mbar_init(&sh.drain, 1);
+    mbar_init(&sh.o_free, ATT_SM_WARPS);
+    mbar_init(&sh.drain, 2);
+    for (int q = 0; q < 4; ++q) mbar_init(&sh.pair_bar[q], 2);
     sh.abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&map_cache);
@@ -274,125 +347,187 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
     if (warp == 0) {
       if (lane == 0) {
         // =========================================================== TMA producer
-        int g = 0;
-        for (int k = 0, s_i = seg_begin; s_i < seg_end; ++k, ++s_i) {
-          const AttnSeg sg = p.segs[s_i];
+        // Two cursors: the score-only chunks run one tile ahead of this CTA's own chunks,
+        // because their slots free up earlier (after S instead of after P·C).
+        auto page_of = [&](const TileCursor& c) {
+          const int b = c.sg.unit / p.n_mt;
+          int page = p.block_table[static_cast<int64_t>(b) * p.max_pages + c.tile];
+          if (page < 0 || page >= p.num_pages) {
+            record_error(MLA_ERR_DEVICE_OOB);
+            page = 0;
+          }
+          return page;
+        };
+        auto load_chunks = [&](const TileCursor& c, int g, bool own, uint64_t* bar) {
+          const int page = page_of(c);
+          uint8_t* st = stage_buf + (g % ATT_STAGES) * ATT_TILE_BYTES;
+          mbar_arrive_expect_tx(bar, (own ? 4 : 5) * ATT_CHUNK_BYTES);
+          for (int j = own ? 5 : 0; j < (own ? 9 : 5); ++j) {
+            const int c_idx = att_chunk_order(half, j);
+            tma_load_2d(st + c_idx * ATT_CHUNK_BYTES, &map_cache, bar, 64 * c_idx,
+                        page * ATT_PAGE);
+          }
+        };
+        auto load_q_smem = [&](const AttnSeg& sg) {   // Q̂[:, 384:576] of a unit
           const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
-          if (k >= 1 && !att_wait(sh, &sh.q_free, (k - 1) & 1)) break;
           mbar_arrive_expect_tx(&sh.q_full, ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES);
-          const int qrow = b * p.R + mt * 128;
           for (int c = 0; c < ATT_QS_CHUNKS; ++c)
             tma_load_2d(qs_buf + c * ATT_QS_CHUNK_BYTES, &map_qhat, &sh.q_full,
-                        ATT_QT_ELEMS + 64 * c, qrow);
-          bool ok = true;
-          for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
-            const int st = g % ATT_STAGES;
-            if (g >= ATT_STAGES && !att_wait(sh, &sh.tile_empty[st], ((g / ATT_STAGES) - 1) & 1)) {
-              ok = false;
-              break;
-            }
-            int page = p.block_table[static_cast<int64_t>(b) * p.max_pages + tile];
-            if (page < 0 || page >= p.num_pages) {
-              record_error(MLA_ERR_DEVICE_OOB);
-              page = 0;
-            }
-            uint8_t* dst = stage_buf + st * ATT_TILE_BYTES;
-            mbar_arrive_expect_tx(&sh.tile_full[st], ATT_TILE_BYTES);
-            for (int c = 0; c < ATT_CHUNKS; ++c)
-              tma_load_2d(dst + c * ATT_CHUNK_BYTES, &map_cache, &sh.tile_full[st], 64 * c,
-                          page * ATT_PAGE);
+                        ATT_QT_ELEMS + 64 * c, b * p.R + mt * 128);
+        };
+        // Step for tile g: its own chunks, then (new segment at g+1) the next Q̂, then the
+        // score-only chunks of tile g+1. Own chunks of g wait for P·C of g-2; score-only chunks
+        // of g+1 wait for S of g-1, which completes earlier, so neither load delays the other.
+        TileCursor cq, co, cp;   // score-only cursor (one tile ahead), own-chunk cursor,
+        cq.init(p.segs, seg_begin, seg_end);   // L2-prefetch cursor (further ahead, half 0 only)
+        co.init(p.segs, seg_begin, seg_end);
+        cp.init(p.segs, seg_begin, seg_end);
+        auto prefetch_next = [&]() {
+          if (half != 0 || !cp.valid()) return;
+          prefetch_l2_bulk(p.cache + static_cast<int64_t>(page_of(cp)) * ATT_PAGE * ATT_ROW,
+                           ATT_TILE_BYTES);
+          cp.next();
+        };
+        for (int i = 0; i < ATT_PREFETCH_AHEAD; ++i) prefetch_next();
+        int gq = 0, go = 0;
+        bool ok = true;
+        load_q_smem(cq.sg);
+        load_chunks(cq, gq, false, &sh.full_qk[0]);
+        cq.next();
+        ++gq;
+        while (ok && co.valid()) {
+          int st = go % ATT_STAGES;
+          if (go >= ATT_STAGES && !att_wait(sh, &sh.empty_own[st], ((go / ATT_STAGES) - 1) & 1)) {
+            ok = false;
+            break;
           }
-          if (!ok) break;
+          load_chunks(co, go, true, &sh.full_own[st]);
+          const bool seg_ends = co.last_of_seg();
+          const int k_done = co.k;
+          co.next();
+          ++go;
+          if (!cq.valid()) continue;
+          if (seg_ends) {   // Q̂ smem of the next segment: the last S of this one must be done
+            if (!att_wait(sh, &sh.q_free, k_done & 1)) { ok = false; break; }
+            load_q_smem(cq.sg);
+          }
+          st = gq % ATT_STAGES;
+          if (gq >= ATT_STAGES && !att_wait(sh, &sh.empty_qk[st], ((gq / ATT_STAGES) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          load_chunks(cq, gq, false, &sh.full_qk[st]);
+          cq.next();
+          ++gq;
+          prefetch_next();
         }
         // drain: the last loads must land before the CTA can exit (bounded, abort or not)
-        for (int j = max(0, g - ATT_STAGES); j < g; ++j)
-          (void)mbar_wait(&sh.tile_full[j % ATT_STAGES], (j / ATT_STAGES) & 1);
+        for (int j = max(0, gq - ATT_STAGES); j < gq; ++j)
+          (void)mbar_wait(&sh.full_qk[j % ATT_STAGES], (j / ATT_STAGES) & 1);
+        for (int j = max(0, go - ATT_STAGES); j < go; ++j)
+          (void)mbar_wait(&sh.full_own[j % ATT_STAGES], (j / ATT_STAGES) & 1);
       }
     } else if (warp == 1) {
       if (lane == 0) {
-        // =========================================================== MMA issuer
-        constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
+        // =========================================================== score MMA issuer
+        const uint32_t stage0 = smem_addr(stage_buf);
+        const uint64_t qs_desc = smem_desc_sw128(smem_addr(qs_buf), 16, 1024);
+        TileCursor cur;
+        cur.init(p.segs, seg_begin, seg_end);
+        for (int g = 0; cur.valid(); ++g, cur.next()) {
+          const int st = g % ATT_STAGES;
+          if (cur.first_of_seg() && !att_wait(sh, &sh.q_full, cur.k & 1)) break;
+          if (g >= 1 && !att_wait(sh, &sh.s_free, (g - 1) & 1)) break;
+          const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
+          // S over the score-only chunks first, then this CTA's own chunks (see att_chunk_order)
+          if (!att_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
+          tc_fence_after_sync();
+          if (half == 0) {
+            att_qk_chunk<0, 0>(tmem, b_stage, qs_desc); att_qk_chunk<0, 1>(tmem, b_stage, qs_desc);
+            att_qk_chunk<0, 2>(tmem, b_stage, qs_desc); att_qk_chunk<0, 3>(tmem, b_stage, qs_desc);
+            att_qk_chunk<0, 4>(tmem, b_stage, qs_desc);
+          } else {
+            att_qk_chunk<1, 0>(tmem, b_stage, qs_desc); att_qk_chunk<1, 1>(tmem, b_stage, qs_desc);
+            att_qk_chunk<1, 2>(tmem, b_stage, qs_desc); att_qk_chunk<1, 3>(tmem, b_stage, qs_desc);
+            att_qk_chunk<1, 4>(tmem, b_stage, qs_desc);
+          }
+          mma_commit(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
+          if (!att_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
+          tc_fence_after_sync();
+          if (half == 0) {
+            att_qk_chunk<0, 5>(tmem, b_stage, qs_desc); att_qk_chunk<0, 6>(tmem, b_stage, qs_desc);
+            att_qk_chunk<0, 7>(tmem, b_stage, qs_desc); att_qk_chunk<0, 8>(tmem, b_stage, qs_desc);
+          } else {
+            att_qk_chunk<1, 5>(tmem, b_stage, qs_desc); att_qk_chunk<1, 6>(tmem, b_stage, qs_desc);
+            att_qk_chunk<1, 7>(tmem, b_stage, qs_desc); att_qk_chunk<1, 8>(tmem, b_stage, qs_desc);
+          }
+          mma_commit(&sh.s_full);
+          if (cur.last_of_seg()) mma_commit(&sh.q_free);
+          mma_commit(&sh.empty_own[st]);
+        }
+        // drain: every MMA issued above completes before TMEM is released
+        mma_commit(&sh.drain);
+        (void)mbar_wait(&sh.drain, 0);
+      }
+    } else if (warp == 6) {
+      if (lane == 0) {
+        // =========================================================== P·C MMA issuer
         constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
         const uint32_t stage0 = smem_addr(stage_buf);
-        const uint32_t qs0 = smem_addr(qs_buf);
-        const uint32_t pb0 = smem_addr(p_buf);
-        int g = 0;            // tile counter over the CTA's segments
-        int pend_g = -1;      // tile whose PV is still to be issued
-        int pend_k = 0;       // its segment counter
-        bool pend_first = false;
-        bool ok = true;
-        auto issue_pv = [&](int gg, int kk_seg, bool first_of_seg) -> bool {
-          if (first_of_seg && kk_seg >= 1 && !att_wait(sh, &sh.o_free, (kk_seg - 1) & 1))
-            return false;
-          if (!att_wait(sh, &sh.p_full, gg & 1)) return false;
+        const uint64_t p_desc = smem_desc_sw128(smem_addr(p_buf), 16, 1024);
+        TileCursor cur;
+        cur.init(p.segs, seg_begin, seg_end);
+        for (int g = 0; cur.valid(); ++g, cur.next()) {
+          const int st = g % ATT_STAGES;
+          const bool first = cur.first_of_seg();
+          if (first && cur.k >= 1 && !att_wait(sh, &sh.o_free, (cur.k - 1) & 1)) break;
+          if (!att_wait(sh, &sh.p_full, g & 1)) break;
           tc_fence_after_sync();
-          const uint32_t st = stage0 + (gg % ATT_STAGES) * ATT_TILE_BYTES +
-                              half * 4 * ATT_CHUNK_BYTES;
+          // O_half += P · C[:, own half]: chunks 4*half .. 4*half+3, read MN-major (N = 256)
+          const uint64_t b0 = smem_desc_sw128(
+              stage0 + st * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES, ATT_CHUNK_BYTES, 1024);
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {   // 16 tokens per K-step
-            mma_bf16_ss(tmem + TM_O, smem_desc_sw128(pb0 + kk * 32, 16, 1024),
-                        smem_desc_sw128(st + kk * 2048, ATT_CHUNK_BYTES, 1024), IDESC_PV,
-                        (first_of_seg && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(&sh.tile_empty[gg % ATT_STAGES]);
+          for (int kk = 0; kk < 4; ++kk)   // 16 tokens per K-step
+            mma_bf16_ss(tmem + TM_O, p_desc + static_cast<uint64_t>(kk * 2),
+                        b0 + static_cast<uint64_t>(kk * 128), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          mma_commit(&sh.empty_own[st]);
           mma_commit(&sh.pv_done);
-          return true;
-        };
-        for (int k = 0, s_i = seg_begin; ok && s_i < seg_end; ++k, ++s_i) {
-          const AttnSeg sg = p.segs[s_i];
-          if (!att_wait(sh, &sh.q_full, k & 1)) { ok = false; break; }
-          for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
-            if (g >= 1 && !att_wait(sh, &sh.s_free, (g - 1) & 1)) { ok = false; break; }
-            if (!att_wait(sh, &sh.tile_full[g % ATT_STAGES], (g / ATT_STAGES) & 1)) { ok = false; break; }
-            tc_fence_after_sync();
-            const uint32_t st = stage0 + (g % ATT_STAGES) * ATT_TILE_BYTES;
-            // S = Q̂ · Cᵀ over 36 K-steps of 16: Q̂[:, 0:384] from TMEM, Q̂[:, 384:576] from smem
-#pragma unroll 4
-            for (int ks = 0; ks < ATT_ROW / 16; ++ks) {
-              const uint64_t bdesc =
-                  smem_desc_sw128(st + (ks >> 2) * ATT_CHUNK_BYTES + (ks & 3) * 32, 16, 1024);
-              if (ks < ATT_QT_ELEMS / 16) {
-                mma_bf16_ts(tmem + TM_S, tmem + TM_Q + ks * 8, bdesc, IDESC_QK, ks > 0 ? 1u : 0u);
-              } else {
-                const int qk = ks - ATT_QT_ELEMS / 16;
-                mma_bf16_ss(tmem + TM_S,
-                            smem_desc_sw128(qs0 + (qk >> 2) * ATT_QS_CHUNK_BYTES + (qk & 3) * 32, 16, 1024),
-                            bdesc, IDESC_QK, 1u);
-              }
-            }
-            mma_commit(&sh.s_full);
-            if (tile + 1 == sg.tile_end) mma_commit(&sh.q_free);
-            if (pend_g >= 0 && !issue_pv(pend_g, pend_k, pend_first)) { ok = false; break; }
-            pend_g = g;
-            pend_k = k;
-            pend_first = (tile == sg.tile_begin);
-          }
         }
-        if (ok && pend_g >= 0) issue_pv(pend_g, pend_k, pend_first);
-        // drain: every MMA issued above completes before TMEM is released
         mma_commit(&sh.drain);
         (void)mbar_wait(&sh.drain, 0);
       }
     } else {
       // ============================================================ softmax warps
+      // Warps 2..5 take score columns 0..31, warps 7..10 columns 32..63 of the same rows.
+      const int hc = warp >= 7 ? 1 : 0;   // column half of the score tile
       const int quarter = warp & 3;
       const int r_local = quarter * 32 + lane;
+      const int t_idx = hc * 128 + r_local;   // 0..255 among the softmax threads
       const uint32_t t_lane = static_cast<uint32_t>(quarter * 32) << 16;
-      int g = 0;
+      int g = 0, xc = 0;   // tile counter, partner-exchange counter
       bool ok = true;
-      // Q̂[:, 0:384] of a unit into TMEM (row r_local), zeros for rows past the unit.
+      // both warps of this lane quarter have published their partial: a bounded meeting
+      auto meet = [&]() -> bool {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.pair_bar[quarter]);
+        const bool r = att_warp_wait(sh, &sh.pair_bar[quarter], xc & 1);
+        ++xc;
+        return r;
+      };
+      // Q̂[:, 0:384] of a unit into TMEM (row r_local), zeros for rows past the unit; each warp
+      // of the pair writes 3 of the 6 column groups.
       auto load_q_tmem = [&](const AttnSeg& sg) {
         const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
         const int r_in = mt * 128 + r_local;
         const bool valid = r_in < p.R;
         const uint4* src = reinterpret_cast<const uint4*>(
             p.qhat + (static_cast<int64_t>(b) * p.R + r_in) * ATT_ROW);
+        uint32_t v[32];
 #pragma unroll 1
-        for (int c = 0; c < ATT_QT_ELEMS / 64; ++c) {
-          uint32_t v[32];
+        for (int c = hc * 3; c < hc * 3 + 3; ++c) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            uint4 x = valid ? src[c * 8 + j] : make_uint4(0, 0, 0, 0);
+            const uint4 x = valid ? src[c * 8 + j] : make_uint4(0, 0, 0, 0);
             v[4 * j + 0] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
           }
           tmem_st32(tmem + t_lane + TM_Q + c * 32, v);
@@ -402,47 +537,54 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.q_full);
       };
-      if (true) load_q_tmem(p.segs[seg_begin]);
+      load_q_tmem(p.segs[seg_begin]);
       for (int k = 0, s_i = seg_begin; ok && s_i < seg_end; ++k, ++s_i) {
         const AttnSeg sg = p.segs[s_i];
         const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
         const int L = p.seq_lens[b];
         const int r_in = mt * 128 + r_local;
         const bool row_valid = r_in < p.R;
-        const int t = row_valid ? r_in / p.H : 0;
-        const int limit = L - p.Tq + t;     // last key this row may see
-        float m_ref = -INFINITY, l_sum = 0.0f;
+        const int limit = L - p.Tq + (row_valid ? r_in / p.H : 0);   // last key this row sees
+        float m_ref = -INFINITY, l_part = 0.0f;
         for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
           if (!att_warp_wait(sh, &sh.s_full, g & 1)) { ok = false; break; }
           tc_fence_after_sync();
-          uint32_t sr[64];
-          {
-            uint32_t (&a)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-            uint32_t (&c)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-            tmem_ld32(tmem + t_lane + TM_S, a);
-            tmem_ld32(tmem + t_lane + TM_S + 32, c);
-          }
+          uint32_t sr[32];
+          tmem_ld32(tmem + t_lane + TM_S + hc * 32, sr);
           tmem_ld_wait();
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.s_free);
-          // masked, base-2 scaled scores and their maximum
-          const int j0 = tile * ATT_PAGE;
+          // this thread's visible columns: 0 .. nvis-1 of its 32
+          const int j0 = tile * ATT_PAGE + hc * 32;
           const int jmax = row_valid ? min(limit, L - 1) : -1;   // inclusive
-          float mt_max = -INFINITY;
+          const int nvis = max(0, min(32, jmax - j0 + 1));
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+          if (nvis == 32) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const float s = (j0 + c <= jmax) ? __uint_as_float(sr[c]) * p.scale_log2 : -INFINITY;
-            sr[c] = __float_as_uint(s);
-            mt_max = fmaxf(mt_max, s);
+            for (int c = 0; c < 32; c += 2) {
+              mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+              mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+            }
+          } else {
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+              mx0 = fmaxf(mx0, c < nvis ? __uint_as_float(sr[c]) : -INFINITY);
+              mx1 = fmaxf(mx1, c + 1 < nvis ? __uint_as_float(sr[c + 1]) : -INFINITY);
+            }
           }
+          // agree on the row maximum with the partner warp (same rows, other 32 columns)
+          sh.row_max[g & 1][hc][r_local] = fmaxf(mx0, mx1);
+          if (!meet()) { ok = false; break; }
+          const float raw_max = fmaxf(sh.row_max[g & 1][0][r_local], sh.row_max[g & 1][1][r_local]);
+          const float mt_max = raw_max > -INFINITY ? raw_max * p.scale_log2 : -INFINITY;
           float factor = 1.0f;
           bool rescale = false;
           if (mt_max > -INFINITY) {
             if (m_ref == -INFINITY) {
               m_ref = mt_max;
             } else if (mt_max > m_ref + ATT_RESCALE_THRESHOLD) {
-              factor = exp2f(m_ref - mt_max);
+              factor = fast_exp2(m_ref - mt_max);
               m_ref = mt_max;
               rescale = true;
             }
@@ -452,7 +594,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           tc_fence_after_sync();
           if (__any_sync(0xffffffffu, rescale) && tile > sg.tile_begin) {
 #pragma unroll 1
-            for (int c0 = 0; c0 < 256; c0 += 32) {
+            for (int c0 = hc * 128; c0 < hc * 128 + 128; c0 += 32) {
               uint32_t o[32];
               tmem_ld32(tmem + t_lane + TM_O + c0, o);
               tmem_ld_wait();
@@ -462,33 +604,41 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
             }
             tmem_st_wait();
           }
-          l_sum *= factor;
-          // P = 2^(s - m_ref) -> bf16, row r_local of the swizzled K-major P tile
-          const float mref_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-          float psum = 0.0f;
+          l_part *= factor;
+          // P = 2^(scale*s - m_ref) -> bf16 (0 for hidden columns), this thread's 4 16-byte
+          // chunks of row r_local of the swizzled K-major P tile
+          const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
+          const float sc = p.scale_log2;
+          float ps0 = 0.0f, ps1 = 0.0f;
           uint8_t* prow = p_buf + r_local * 128;
 #pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {
+          for (int q = 0; q < 4; ++q) {
             uint32_t w[4];
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float x0 = exp2f(__uint_as_float(sr[ch * 8 + 2 * e]) - mref_use);
-              const float x1 = exp2f(__uint_as_float(sr[ch * 8 + 2 * e + 1]) - mref_use);
-              psum += x0 + x1;
+              const int c = q * 8 + 2 * e;
+              float x0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
+              float x1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
+              if (nvis < 32) {
+                x0 = c < nvis ? x0 : 0.0f;
+                x1 = c + 1 < nvis ? x1 : 0.0f;
+              }
+              ps0 += x0;
+              ps1 += x1;
               w[e] = pack_bf16x2(x0, x1);
             }
+            const int ch = hc * 4 + q;
             *reinterpret_cast<uint4*>(prow + ((ch ^ (r_local & 7)) * 16)) =
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
-          l_sum += psum;
+          l_part += ps0 + ps1;
           // rows past the sequence end must be zero in the value chunks (P is 0 there, but
-          // stale cache contents could be non-finite)
-          const int valid_tok = L - j0;
+          // stale cache contents could be non-finite); S is done, so they have landed
+          const int valid_tok = L - tile * ATT_PAGE;
           if (valid_tok < ATT_PAGE) {
-            if (!att_warp_wait(sh, &sh.tile_full[g % ATT_STAGES], (g / ATT_STAGES) & 1)) { ok = false; break; }
             uint8_t* vbase = stage_buf + (g % ATT_STAGES) * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES;
             const int nrows = ATT_PAGE - valid_tok;
-            for (int i = r_local; i < 4 * nrows * 8; i += 128) {
+            for (int i = t_idx; i < 4 * nrows * 8; i += 256) {
               const int chunk = i / (nrows * 8);
               const int rem = i % (nrows * 8);
               const int row = valid_tok + rem / 8, piece = rem % 8;
@@ -509,13 +659,16 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           tc_fence_after_sync();
           load_q_tmem(p.segs[s_i + 1]);
         }
-        // segment epilogue: O / l and the log-sum-exp
+        // segment epilogue: O / l (this thread's 128 of the CTA's 256 columns) and the lse
+        sh.row_sum[hc][r_local] = l_part;
+        if (!meet()) { ok = false; break; }
+        const float l_sum = sh.row_sum[0][r_local] + sh.row_sum[1][r_local];
         if (!att_warp_wait(sh, &sh.pv_done, seg_last_g & 1)) { ok = false; break; }
         tc_fence_after_sync();
         const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
         float* dst = p.o_part + (static_cast<int64_t>(s_i) * 128 + r_local) * ATT_DC + half * 256;
 #pragma unroll 1
-        for (int c0 = 0; c0 < 256; c0 += 32) {
+        for (int c0 = hc * 128; c0 < hc * 128 + 128; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tmem + t_lane + TM_O + c0, o);
           tmem_ld_wait();
@@ -525,7 +678,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                 make_float4(__uint_as_float(o[j]) * inv_l, __uint_as_float(o[j + 1]) * inv_l,
                             __uint_as_float(o[j + 2]) * inv_l, __uint_as_float(o[j + 3]) * inv_l);
         }
-        if (half == 0)
+        if (half == 0 && hc == 0)
           p.lse[static_cast<int64_t>(s_i) * 128 + r_local] =
               (l_sum > 0.0f) ? m_ref + log2f(l_sum) : -INFINITY;
         tc_fence_before_sync();

@@ -104,11 +104,12 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
       }
       tc_fence_after_sync();
       const uint32_t sa = smem_addr(smem + s * STAGE_BYTES);
-      const uint32_t sb = sa + A_BYTES;
+      const uint64_t a0 = smem_desc_sw128(sa, 16, 1024);
+      const uint64_t b0 = smem_desc_sw128(sa + A_BYTES, 16, 1024);
 #pragma unroll
-      for (int kk = 0; kk < GEMM_BK / 16; ++kk) {
-        mma_bf16_ss(tmem, smem_desc_sw128(sa + kk * 32, 16, 1024),
-                    smem_desc_sw128(sb + kk * 32, 16, 1024), IDESC, (i > 0 || kk > 0) ? 1u : 0u);
+      for (int kk = 0; kk < GEMM_BK / 16; ++kk) {   // +32 bytes per K-step of 16
+        mma_bf16_ss(tmem, a0 + static_cast<uint64_t>(kk * 2), b0 + static_cast<uint64_t>(kk * 2), IDESC,
+                    (i > 0 || kk > 0) ? 1u : 0u);
       }
       mma_commit(&empty_bar[s]);
     }

@@ -137,8 +137,9 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t t
  *   w_uk_t      [n_heads, d_c, d_nope], w_uv [n_heads, d_v, d_c]   (from mla_absorb_weights)
  *   workspace   >= mla_decode_workspace_size(cfg, batch, tq) bytes, 256-byte aligned
  *   out         [batch, tq, n_heads, d_v]
- * bf16 runs on the tcgen05 tensor-core path and needs d_c = 512, d_rope = 64, d_nope = 128,
- * d_v = 128, page_size = 64 (DeepSeek-V2 shapes); fp32 runs on CUDA cores for any shape.
+ * bf16 runs on the tcgen05 tensor-core path and needs d_c = 512, d_rope = 64, page_size = 64
+ * and d_nope a multiple of 64 (DeepSeek-V2 latent shapes); fp32 runs on CUDA cores for any
+ * shape.
  * A sequence whose length is out of range gets zero output and MLA_ERR_DEVICE_BAD_LENGTH.
  */
 mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
@@ -146,6 +147,22 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
                       int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
                       const void* w_uv, void* workspace, size_t ws_bytes, void* out,
                       void* stream);
+
+/*
+ * mla_decode with per-kernel timing: identical arguments and results, plus `events`, an array
+ * of 6 cudaEvent_t created by the caller. events[i] is recorded on `stream` just before decode
+ * kernel i (0 planning, 1 query absorption, 2 latent attention, 3 split combine, 4 value
+ * projection) and events[5] after the last one, so cudaEventElapsedTime(events[2], events[3])
+ * is the attention kernel's device time. While `stream` is being captured the events are
+ * recorded with cudaEventRecordExternal, so they become event-record nodes of the graph. On the fp32 path, which
+ * has no planning or combine kernel, events 0/1 mark the start and 3/4 the end of attention.
+ * NULL entries are skipped.
+ */
+mla_status mla_decode_profiled(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                               const void* cache, int32_t num_pages, const int32_t* block_table,
+                               int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                               const void* w_uv, void* workspace, size_t ws_bytes, void* out,
+                               void* stream, void* const* events);
 
 /* Bytes of workspace mla_prefill_ref needs (0 if the arguments are invalid). */
 size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new);
