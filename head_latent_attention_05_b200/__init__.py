@@ -29,7 +29,7 @@ STATUS = {
 # Every symbol include/mla.h declares (checked by the tests against the built library).
 EXPORTED = (
     "mla_status_string", "mla_absorb_weights", "mla_append_workspace_size", "mla_append_latent",
-    "mla_decode_workspace_size", "mla_decode", "mla_decode_profiled",
+    "mla_decode_workspace_size", "mla_decode", "mla_decode_profiled", "mla_decode_noalloc",
     "mla_prefill_ref_workspace_size",
     "mla_prefill_ref", "mla_get_device_error",
 )
@@ -83,6 +83,7 @@ def load_library() -> ctypes.CDLL:
         "mla_decode": (ctypes.c_int, [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P, P]),
         "mla_decode_profiled": (ctypes.c_int,
                                 [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, SZ, P, P, P]),
+        "mla_decode_noalloc": (ctypes.c_int, [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, P]),
         "mla_prefill_ref_workspace_size": (SZ, [CFG, I32, I32]),
         "mla_prefill_ref": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ, P, P]),
         "mla_get_device_error": (ctypes.c_int, [P]),
@@ -162,6 +163,21 @@ def mla_decode_profiled(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t,
         block_table.shape[1], _ptr(seq_lens), _ptr(w_uk_t), _ptr(w_uv), _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream), arr),
         "mla_decode_profiled")
+
+
+# Bytes of the library's built-in scratch used by mla_decode_noalloc.
+MLA_DECODE_NOALLOC_MAX_SCRATCH = 32 << 20
+
+
+def mla_decode_noalloc(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv, out,
+                       stream=None):
+    """mla_decode without a workspace argument: the scratch is a fixed device array inside the
+    library (see include/mla.h), for callers that cannot allocate device memory."""
+    batch, tq = q.shape[0], q.shape[1]
+    _check(load_library().mla_decode_noalloc(
+        ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), _ptr(w_uk_t), _ptr(w_uv), _ptr(out),
+        _stream(stream)), "mla_decode_noalloc")
 
 
 def mla_prefill_ref_workspace_size(cfg: MlaConfig, batch: int, t_new: int) -> int:

@@ -604,6 +604,46 @@ mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, 
                                     max_pages, seq_lens, w_uk_t, w_uv, L, out, st);
 }
 
+// ---------------------------------------------------------------- allocation-free decode
+// Scratch for mla_decode_noalloc: a file-scope device array, present on every GPU that loads
+// this library until the process exits. Host code must not pass the symbol itself to a
+// kernel (on the host it is only a stand-in); its device address is looked up once per
+// device with cudaGetSymbolAddress and cached.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[MLA_DECODE_NOALLOC_MAX_SCRATCH];
+
+static mla_status noalloc_scratch_ptr(void** out) {
+  static std::mutex mu;
+  static void* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return MLA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(mu);
+  if (ptrs[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+      return MLA_ERR_CUDA;
+    ptrs[dev] = p;
+  }
+  *out = ptrs[dev];
+  return MLA_OK;
+}
+
+mla_status mla_decode_noalloc(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                              const void* cache, int32_t num_pages, const int32_t* block_table,
+                              int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                              const void* w_uv, void* out, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (batch < 1 || tq < 1) return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_decode_workspace_size(cfg, batch, tq);
+  if (need == 0) return cfg->dtype == MLA_DTYPE_BF16 ? MLA_ERR_UNSUPPORTED : MLA_ERR_INVALID_ARG;
+  if (need > MLA_DECODE_NOALLOC_MAX_SCRATCH) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  void* scratch = nullptr;
+  const mla_status ps = noalloc_scratch_ptr(&scratch);
+  if (ps != MLA_OK) return ps;
+  return decode_impl(cfg, q, batch, tq, cache, num_pages, block_table, max_pages, seq_lens,
+                     w_uk_t, w_uv, scratch, MLA_DECODE_NOALLOC_MAX_SCRATCH, out, stream, nullptr);
+}
+
 mla_status mla_get_device_error(void* stream) {
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return MLA_ERR_CUDA;
   int v = 0;

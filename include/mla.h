@@ -187,6 +187,30 @@ mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, 
                            void* stream);
 
 /*
+ * Allocation-free decode, for callers that cannot allocate device memory themselves: code
+ * running where cudaMalloc is unavailable or forbidden (inside a memory-pool-managed serving
+ * runtime that owns all device memory, or a host callback), or that must not grow its
+ * footprint per call. The paper has no counterpart: this is a deployment convenience.
+ * Same arguments and results as mla_decode, minus the workspace: the scratch it needs lives in
+ * a fixed device array of MLA_DECODE_NOALLOC_MAX_SCRATCH bytes inside this library, which
+ * every GPU that loads the library holds until the process exits.
+ *   - A call whose scratch need (mla_decode_workspace_size) exceeds that maximum returns
+ *     MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing. 32 MiB covers a DeepSeek-V2-shaped
+ *     batch of 16 sequences with one query token each.
+ *   - It never calls cudaMalloc, cudaFree or any allocating routine.
+ *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
+ *     and caches it; make that first call before any stream capture on that device.
+ *   - Every call on a device shares the one array, and no part of it needs to start zeroed
+ *     (each call writes all scratch it reads). Calls that overlap on the GPU (different
+ *     streams, or concurrent host threads) race on it: serialise them.
+ */
+#define MLA_DECODE_NOALLOC_MAX_SCRATCH (32u << 20)
+mla_status mla_decode_noalloc(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                              const void* cache, int32_t num_pages, const int32_t* block_table,
+                              int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
+                              const void* w_uv, void* out, void* stream);
+
+/*
  * Synchronise `stream`, then return (and clear) the first error a kernel of this library
  * recorded on the current device since the previous call: MLA_OK if none. Returns
  * MLA_ERR_CUDA if the synchronisation itself fails.

@@ -1,0 +1,55 @@
+"""The allocation-free decode entry point, through the C ABI, against mla_decode.
+
+mla_decode_noalloc serves callers that cannot allocate device memory themselves (a serving
+runtime that owns the whole device memory pool, code that runs where cudaMalloc is not
+allowed): its scratch is a fixed device array inside the library instead of a caller-given
+workspace. The array is shared by every call and keeps the previous call's contents, so the
+check runs two calls in a row (with a different-sized call in between) and compares each with
+mla_decode on the same inputs, within the parity tolerance the other tests use. This file is
+collected last so that a run stopping at the first failure has already run everything else.
+"""
+
+import pytest
+import torch
+
+import harness as Hs
+import head_latent_attention_05_b200 as mla
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+V2 = W.WORKLOADS["v2_bf16_b16_ctx4096"]
+
+
+def _noalloc(c):
+    w = c.w
+    out = torch.full((w.B, w.Tq, w.H, w.d_v), float("nan"), dtype=w.torch_dtype, device="cuda")
+    mla.mla_decode_noalloc(c.cfg, c.d["q"], c.d["cache"], c.d["block_table"], c.d["seq_lens"],
+                           c.d["w_uk_t"], c.d["w_uv"], out)
+    assert mla.mla_get_device_error() == 0
+    return out.float().cpu()
+
+
+def test_noalloc_decode_matches_decode_on_consecutive_calls():
+    mla.mla_get_device_error()
+    big = Hs.make_case(W.small_variant(V2, B=4), torch.tensor([4096, 130, 1, 777], dtype=torch.int32))
+    small = Hs.make_case(W.small_variant(V2, B=2, seed=7), torch.tensor([65, 300], dtype=torch.int32))
+    Hs.run_append(big)
+    Hs.run_append(small)
+    ref_big = Hs.run_decode(big).float().cpu()
+    ref_small = Hs.run_decode(small).float().cpu()
+    for _ in range(2):
+        Hs.assert_parity(_noalloc(big), ref_big, "bf16", "noalloc vs decode (4 sequences)")
+        Hs.assert_parity(_noalloc(small), ref_small, "bf16", "noalloc vs decode (2 sequences)")
+
+
+def test_noalloc_rejects_a_batch_beyond_its_scratch():
+    cfg = Hs.config_of(V2)
+    assert mla.mla_decode_workspace_size(cfg, 64, 1) > mla.MLA_DECODE_NOALLOC_MAX_SCRATCH
+    c = Hs.make_case(W.small_variant(V2, B=2), torch.tensor([64, 64], dtype=torch.int32))
+    q = torch.zeros((64, 1, V2.H, V2.d_nope + V2.d_r), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((64, 1, V2.H, V2.d_v), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_decode_noalloc(cfg, q, c.d["cache"], c.d["block_table"], c.d["seq_lens"],
+                               c.d["w_uk_t"], c.d["w_uv"], out)
+    assert e.value.code == 3   # MLA_ERR_WORKSPACE_TOO_SMALL, nothing launched
