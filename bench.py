@@ -4,15 +4,19 @@
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 
 A step is one pass of the whole hot path over one batch of synthetic input:
-mla_append_latent (down-projection GEMM + RMSNorm/RoPE/scatter) then mla_decode (plan, query
-absorption, latent attention, split combine, value projection), through the C ABI. The metric
+mla_append_latent (down-projection GEMM + RMSNorm/RoPE/scatter) then mla_decode (query
+absorption with the split-KV planner, latent attention, split merge fused with the value
+projection), five kernel launches through the C ABI. The metric
 is cache-tokens x heads per second: sum_b L_b * Tq * H / step time, summed over all GPUs
 (each GPU decodes its own batch: weak scaling, no data-path collective).
 
 Timing: the K timed steps are captured once into a CUDA graph (so host launch latency stays
 out of device time) and replayed; before every step the graph writes 256 MiB to flush the
-126 MB L2, outside the step's CUDA events. Per-kernel times come from events the library
-records at its kernel boundaries. `e2e` repeats the step through the plain API from pinned
+126 MB L2, outside the step's CUDA events, which bracket each step and nothing inside it.
+Per-kernel times (and the attention kernel's time in the roofline) come from a second replay
+of the same steps in which the library records events between its kernels (those marks stop
+consecutive kernels from overlapping their start and end, so they are not in the headline).
+`e2e` repeats the step through the plain API from pinned
 host buffers, with the host->device copies of the step's inputs and the device->host copy of
 its output inside the timed region. rank 0 prints one JSON line.
 """
@@ -253,23 +257,29 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     K, Wm = args.steps, max(3, args.warmup)
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
-    step_ev = [[ev() for _ in range(8)] for _ in range(K)]   # start, 6 decode marks, end
+    # headline: one start and one end event per step, nothing between the kernels
+    step_ev = [[ev() for _ in range(2)] for _ in range(K)]
+    # breakdown replay: start, the 4 decode marks (absorption, attention, merge+projection, end)
+    prof_ev = [[ev() for _ in range(5)] for _ in range(K)]
     # torch creates events lazily: record every event once so it exists before capture
-    for evs in step_ev:
+    for evs in step_ev + prof_ev:
         for e in evs:
             e.record()
     torch.cuda.synchronize()
 
-    def step(evs=None):
+    def step(evs=None, marks=None):
         if evs is not None:
             evs[0].record()
+        if marks is not None:
+            marks[0].record()
         mla.mla_append_latent(cfg, x_new, w_dkv, kv_gain, seq_idx, pos, bt, cache, ws_a)
-        if evs is not None:
+        if marks is not None:
             mla.mla_decode_profiled(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out,
-                                    evs[1:7])
-            evs[7].record()
+                                    marks[1:5])
         else:
             mla.mla_decode(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out)
+        if evs is not None:
+            evs[1].record()
 
     # warm-up (eager), then a correctness guard: no device error may be pending
     for i in range(Wm):
@@ -279,18 +289,31 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if err != 0:
         raise RuntimeError(f"device error during warm-up: {mla.mla_status_string(err)}")
 
-    graph = None
-    if not args.no_graph:
-        graph = torch.cuda.CUDAGraph()
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
         s = torch.cuda.Stream(device=dev)
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
-            with torch.cuda.graph(graph, stream=s):
-                for i in range(K):
-                    flush.fill_((i * 7) & 0xFF)
-                    step(step_ev[i])
+            with torch.cuda.graph(g, stream=s):
+                fn()
         torch.cuda.current_stream().wait_stream(s)
         torch.cuda.synchronize()
+        return g
+
+    def timed_steps():
+        for i in range(K):
+            flush.fill_((i * 7) & 0xFF)
+            step(evs=step_ev[i])
+
+    def marked_steps():
+        for i in range(K):
+            flush.fill_((i * 7) & 0xFF)
+            step(marks=prof_ev[i])
+
+    graph = graph_prof = None
+    if not args.no_graph:
+        graph = capture(timed_steps)
+        graph_prof = capture(marked_steps)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -302,9 +325,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if graph is not None:
         graph.replay()
     else:
-        for i in range(K):
-            flush.fill_((i * 7) & 0xFF)
-            step(step_ev[i])
+        timed_steps()
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
     if world > 1:
@@ -313,12 +334,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     err = mla.mla_get_device_error()
     if err != 0:
         raise RuntimeError(f"device error in the timed region: {mla.mla_status_string(err)}")
+    # the breakdown replay (same steps, event marks between the kernels)
+    if graph_prof is not None:
+        graph_prof.replay()
+    else:
+        marked_steps()
+    torch.cuda.synchronize()
 
-    names = ["append", "plan", "q_absorb", "attention", "combine", "value_proj"]
+    names = ["append", "q_absorb_plan", "attention", "merge_value_proj"]
     per = {n: [] for n in names}
-    steps_ms = []
-    for evs in step_ev:
-        steps_ms.append(evs[0].elapsed_time(evs[7]))
+    steps_ms = [evs[0].elapsed_time(evs[1]) for evs in step_ev]
+    for evs in prof_ev:
         for j, n in enumerate(names):
             per[n].append(evs[j].elapsed_time(evs[j + 1]))
     total_ms = sum(steps_ms)
@@ -329,6 +355,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     ms_per_step = total_ms / K
     value = world * work["units"] / (ms_per_step / 1e3)
     kernel_ms = {n: statistics.fmean(v) for n, v in per.items()}
+    kernel_ms["marked_step"] = statistics.fmean(
+        evs[0].elapsed_time(evs[4]) for evs in prof_ev)
 
     # ---- e2e through the plain API from pinned host buffers
     x_pin = x_new_h.contiguous().pin_memory()
@@ -402,13 +430,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "heads": w.H, "tq": w.Tq, "context": list(w.lens),
                    "cache_tokens_per_gpu": work["tokens"], "parallelism": f"dp{world}",
                    "l2": "flushed before every step (256 MiB write, outside the step events)",
-                   "timing": "CUDA graph of the K steps" if graph is not None else "eager",
+                   "timing": ("CUDA graph of the K steps" if graph is not None else "eager")
+                   + "; kernel_ms and the roofline's kernel time from a second replay of the same"
+                   " steps with event marks between the kernels",
                    "step": "mla_append_latent + mla_decode"},
         "roofline": roof,
         "kernel_ms": kernel_ms,
         "e2e": {"value": world * work["units"] / (e2e_step / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step},
-        "gpu_launches": K * 7,
+        "gpu_launches": K * 5,
         "clocks": clk,
         "wall_s_timed_region": t_wall,
     }
@@ -420,7 +450,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                 "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph
+    del graph, graph_prof
 
 
 def kernel_sha() -> str:

@@ -150,13 +150,14 @@ def mla_decode(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv, wo
 
 def mla_decode_profiled(cfg: MlaConfig, q, cache, block_table, seq_lens, w_uk_t, w_uv,
                         workspace, out, events, stream=None):
-    """mla_decode that also records 6 torch.cuda.Event objects at its kernel boundaries.
+    """mla_decode that also records 4 torch.cuda.Event objects at its kernel boundaries
+    (before the query absorption, the attention, the merge + value projection, and after).
 
     The events must already exist on the device (torch creates them lazily: record each once
     before the first call). Create them with external=True to time inside a CUDA graph."""
-    if len(events) != 6 or any(e.cuda_event == 0 for e in events):
-        raise ValueError("mla_decode_profiled needs 6 already-created CUDA events")
-    arr = (ctypes.c_void_p * 6)(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    if len(events) != 4 or any(e.cuda_event == 0 for e in events):
+        raise ValueError("mla_decode_profiled needs 4 already-created CUDA events")
+    arr = (ctypes.c_void_p * 4)(*[ctypes.c_void_p(e.cuda_event) for e in events])
     batch, tq = q.shape[0], q.shape[1]
     _check(load_library().mla_decode_profiled(
         ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),

@@ -79,17 +79,32 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+constexpr int MLA_MAX_ROPE_PAIRS = 64;   // d_rope <= 128
+
+// Per rotary pair i, f_i = theta^(-2i/d_rope) / pi split into two floats (f_hi + f_lo carries
+// f_i to ~48 bits), formed on the host in double precision and passed to the kernels by value.
+struct RopeFreqs {
+  float f_hi[MLA_MAX_ROPE_PAIRS];
+  float f_lo[MLA_MAX_ROPE_PAIRS];
+};
+
 // RoPE of one pair (x, y) = (v[2i], v[2i+1]) at position pos: turn by pos * theta^(-2i/d).
-// The angle is formed in double precision and reduced to [-pi, pi] there, so that positions
-// up to 2^17 keep full fp32 accuracy; the rotation itself is done in fp32.
-__device__ __forceinline__ void rope_pair(float x, float y, int pair, int d, int pos,
-                                          float theta, float* ox, float* oy) {
-  const double two_pi = 6.283185307179586476925286766559;
-  const double inv_freq = exp2(-(2.0 * pair / static_cast<double>(d)) * log2(static_cast<double>(theta)));
-  const double ang = static_cast<double>(pos) * inv_freq;
-  const float r = static_cast<float>(ang - two_pi * rint(ang / two_pi));
+// In units of pi the angle is t = pos * f_i. pos is split into a = pos with its low 12 bits
+// cleared and b = its low 12 bits (both exact in fp32); each product with f_hi is formed exactly
+// as a rounded value plus its fma residual, the rounded parts are reduced modulo 2 (exact: they
+// are within 1 of an even integer, or are even integers themselves), and sinpi/cospi take the
+// small remainder. Everything stays in fp32 (fp64 is slow on the device), and for positions up
+// to 2^30 the angle keeps an absolute error of about 1e-6 rad.
+__device__ __forceinline__ void rope_pair(float x, float y, float f_hi, float f_lo, int pos,
+                                          float* ox, float* oy) {
+  const float a = static_cast<float>(pos & ~0xFFF), b = static_cast<float>(pos & 0xFFF);
+  const float p1 = a * f_hi, e1 = fmaf(a, f_hi, -p1);
+  const float p2 = b * f_hi, e2 = fmaf(b, f_hi, -p2);
+  const float r1 = p1 - 2.0f * rintf(0.5f * p1);
+  const float r2 = p2 - 2.0f * rintf(0.5f * p2);
+  const float t = (r1 + r2) + ((e1 + e2) + fmaf(a, f_lo, b * f_lo));
   float s, c;
-  sincosf(r, &s, &c);
+  sincospif(t, &s, &c);
   *ox = x * c - y * s;
   *oy = x * s + y * c;
 }

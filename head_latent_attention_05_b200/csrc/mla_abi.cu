@@ -18,6 +18,7 @@
 #include "simt.cuh"
 #include "tc_decode.cuh"
 #include "tc_gemm.cuh"
+#include "tc_vproj.cuh"
 
 using namespace mla;
 
@@ -55,7 +56,21 @@ mla_status check_config(const mla_config* c) {
   // every row must stay 16-byte aligned for vector loads and TMA
   const int64_t row_bytes = static_cast<int64_t>(c->d_c + c->d_rope) * elem_bytes(c);
   if (row_bytes % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  if (c->d_rope > 2 * MLA_MAX_ROPE_PAIRS) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
+}
+
+// theta^(-2i/d_rope) / pi per rotary pair, in double precision on the host, split hi + lo.
+RopeFreqs rope_freqs(const mla_config* c) {
+  RopeFreqs f{};
+  const double pi = 3.141592653589793238462643383279502884;
+  for (int i = 0; i < c->d_rope / 2 && i < MLA_MAX_ROPE_PAIRS; ++i) {
+    const double v = std::pow(static_cast<double>(c->rope_theta),
+                              -2.0 * static_cast<double>(i) / static_cast<double>(c->d_rope)) / pi;
+    f.f_hi[i] = static_cast<float>(v);
+    f.f_lo[i] = static_cast<float>(v - static_cast<double>(f.f_hi[i]));
+  }
+  return f;
 }
 
 // The bf16 decode path: tcgen05 kernels written for DeepSeek-V2 latent shapes.
@@ -73,6 +88,41 @@ int device_sm_count() {
 
 mla_status last_launch_status() {
   return cudaGetLastError() == cudaSuccess ? MLA_OK : MLA_ERR_CUDA;
+}
+
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel of the stream finishes, and calls pdl_wait() before it reads that kernel's output.
+// Used only for the second and later kernels of one call, whose predecessor is the library's
+// own kernel (which triggers only after its own wait).
+// cluster_x > 1 also launches the grid as clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+mla_status launch_pdl_clustered(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                cudaStream_t st, unsigned cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.numAttrs = 1;
+  if (cluster_x > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster_x;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  cfg.attrs = attr;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess
+             ? MLA_OK
+             : MLA_ERR_CUDA;
+}
+template <typename... KArgs, typename... Args>
+mla_status launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                      cudaStream_t st, Args&&... args) {
+  return launch_pdl_clustered(kernel, grid, block, smem, st, 1u, std::forward<Args>(args)...);
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda).
@@ -158,17 +208,20 @@ template <int BN, class Epi>
 mla_status launch_gemm_bn(const CUtensorMap& A, const CUtensorMap& B, const GemmShape& shp,
                           int m_tiles, int Z, const Epi& epi, cudaStream_t st) {
   auto kern = gemm_tc_kernel<BN, Epi>;
-  constexpr int smem = gemm_smem_bytes<BN>();
+  constexpr int smem = gemm_smem_bytes<BN, Epi>();
+  if (shp.m_per_cta < 1 || gemm_tmem_cols(BN, shp.m_per_cta) > 512) return MLA_ERR_UNSUPPORTED;
   if (!allow_smem(kern, smem)) return MLA_ERR_CUDA;
-  const dim3 grid(m_tiles, (shp.N + BN - 1) / BN, Z * shp.k_splits);
+  const dim3 grid((m_tiles + shp.m_per_cta - 1) / shp.m_per_cta, (shp.N + BN - 1) / BN,
+                  Z * shp.k_splits + shp.aux_blocks);
   kern<<<grid, 128, smem, st>>>(A, B, shp, epi);
   return last_launch_status();
 }
 
+// bn: the activation tile (16..256; pick_bn(N) unless a caller caps it).
 template <class Epi>
 mla_status launch_gemm(const CUtensorMap& A, const CUtensorMap& B, const GemmShape& shp,
-                       int m_tiles, int Z, const Epi& epi, cudaStream_t st) {
-  switch (pick_bn(shp.N)) {
+                       int m_tiles, int Z, const Epi& epi, cudaStream_t st, int bn) {
+  switch (bn) {
     case 16: return launch_gemm_bn<16>(A, B, shp, m_tiles, Z, epi, st);
     case 32: return launch_gemm_bn<32>(A, B, shp, m_tiles, Z, epi, st);
     case 64: return launch_gemm_bn<64>(A, B, shp, m_tiles, Z, epi, st);
@@ -211,7 +264,7 @@ struct DecodeLayout {
   int P, n_mt, R, U, max_segs;
   int32_t *unit_tiles, *unit_seg, *pair_seg;
   AttnSeg* segs;
-  __nv_bfloat16 *qhat, *o_lat;
+  __nv_bfloat16* qhat;
   float *o_part, *lse;
   size_t bytes;
 };
@@ -220,7 +273,8 @@ struct DecodeLayout {
 // an SM), two CTAs per pair.
 int attn_pairs() {
   const int sms = device_sm_count();
-  return (sms >= 2 ? sms : 2) / 2;
+  const int pairs = (sms >= 2 ? sms : 2) / 2;
+  return pairs < ATT_MAX_PAIRS ? pairs : ATT_MAX_PAIRS;
 }
 
 DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
@@ -236,7 +290,6 @@ DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
   L.pair_seg = cv.take<int32_t>(L.P + 1);
   L.segs = cv.take<AttnSeg>(L.max_segs);
   L.qhat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_ROW);
-  L.o_lat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_DC);
   L.o_part = cv.take<float>(static_cast<size_t>(L.max_segs) * 128 * ATT_DC);
   L.lse = cv.take<float>(static_cast<size_t>(L.max_segs) * 128);
   L.bytes = cv.off;
@@ -278,15 +331,14 @@ mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const 
   const int max_pos = max_pages * c->page_size;
   qabs_simt_kernel<T><<<rows, 256, (c->d_nope + c->d_rope) * sizeof(float), st>>>(
       static_cast<const T*>(q), static_cast<const T*>(w_uk_t), seq_lens, L.qhat, c->n_heads,
-      Tq, c->d_c, c->d_rope, c->d_nope, max_pos, c->rope_theta);
+      Tq, c->d_c, c->d_rope, c->d_nope, max_pos, rope_freqs(c));
   const int attn_smem = (row + c->d_c) * static_cast<int>(sizeof(float));
   if (!allow_smem(attn_simt_kernel<T>, attn_smem)) return MLA_ERR_CUDA;
-  mark(2);
+  mark(1);
   attn_simt_kernel<T><<<rows, 256, attn_smem, st>>>(
       L.qhat, static_cast<const T*>(cache), block_table, seq_lens, L.o_lat, c->n_heads, Tq,
       c->d_c, c->d_rope, max_pages, num_pages, c->page_size, c->softmax_scale);
-  mark(3);
-  mark(4);
+  mark(2);
   outproj_simt_kernel<T><<<rows, 256, c->d_c * sizeof(float), st>>>(
       L.o_lat, static_cast<const T*>(w_uv), static_cast<T*>(out), c->n_heads, c->d_c, c->d_v);
   return last_launch_status();
@@ -305,7 +357,7 @@ mla_status simt_append(const mla_config* c, const void* x, int n_tok, const void
   append_finish_kernel<T><<<n_tok, finish_threads(row), row * sizeof(float), st>>>(
       kv, 1, n_tok, static_cast<const T*>(kv_gain), seq_idx, pos, block_table, batch,
       max_pages, static_cast<T*>(cache), num_pages, c->page_size, c->d_c, c->d_rope,
-      c->rms_eps, c->rope_theta);
+      c->rms_eps, rope_freqs(c));
   return last_launch_status();
 }
 
@@ -408,15 +460,20 @@ mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok
     if (!make_map(&mB, x, 3, dims, strides, box)) return MLA_ERR_CUDA;
   }
   float* partial = static_cast<float*>(workspace);
-  GemmShape shp{row, n_tok, ap.k_chunks, ap.chunks_per_split, ap.k_splits, 0};
+  GemmShape shp{row, n_tok, ap.k_chunks, ap.chunks_per_split, ap.k_splits, 0, 1, 0};
   EpiSplitK epi{partial, n_tok, row};
-  mla_status s = launch_gemm(mA, mB, shp, ap.m_tiles, 1, epi, st);
+  mla_status s = launch_gemm(mA, mB, shp, ap.m_tiles, 1, epi, st, pick_bn(n_tok));
   if (s != MLA_OK) return s;
-  append_finish_kernel<__nv_bfloat16><<<n_tok, finish_threads(row), row * sizeof(float), st>>>(
-      partial, ap.k_splits, n_tok, static_cast<const __nv_bfloat16*>(kv_gain), seq_idx, pos,
-      block_table, batch, max_pages, static_cast<__nv_bfloat16*>(cache), num_pages,
-      cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps, cfg->rope_theta);
-  return last_launch_status();
+  // the finish runs as clusters of FIN_CLUSTER CTAs per token (see append_finish_cluster_kernel)
+  const int per = (((row + FIN_CLUSTER - 1) / FIN_CLUSTER) + 1) & ~1;
+  return launch_pdl_clustered(append_finish_cluster_kernel<__nv_bfloat16>,
+                              dim3(static_cast<unsigned>(n_tok) * FIN_CLUSTER), dim3(FIN_THREADS),
+                              per * sizeof(float), st, FIN_CLUSTER,
+                              static_cast<const float*>(partial), ap.k_splits, n_tok,
+                              static_cast<const __nv_bfloat16*>(kv_gain), seq_idx, pos,
+                              block_table, batch, max_pages, static_cast<__nv_bfloat16*>(cache),
+                              num_pages, cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps,
+                              rope_freqs(cfg));
 }
 
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq) {
@@ -443,8 +500,8 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
   if (cfg->dtype == MLA_DTYPE_BF16 && !tc_decode_shape(cfg)) return MLA_ERR_UNSUPPORTED;
   if (ws_bytes < mla_decode_workspace_size(cfg, batch, tq)) return MLA_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  // events[i] (if given) is recorded before kernel i: plan, q absorption, attention, combine,
-  // value projection; events[5] after the last one.
+  // events[i] (if given): [0] before the query absorption (which also plans the split-KV
+  // work), [1] before the attention kernel, [2] before the merge + value projection, [3] after.
   auto mark = [&](int i) {
     if (events != nullptr && events[i] != nullptr)
       record_mark(static_cast<cudaEvent_t>(events[i]), st);
@@ -453,11 +510,10 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
   if (cfg->dtype == MLA_DTYPE_F32) {
     const SimtLayout L = simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, workspace);
     mark(0);
-    mark(1);
     const mla_status s = simt_decode<float>(cfg, q, batch, tq, cache, num_pages, block_table,
                                             max_pages, seq_lens, w_uk_t, w_uv, L, out, st,
                                             events);
-    mark(5);
+    mark(3);
     return s;
   }
 
@@ -467,14 +523,10 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
   const int max_pos = max_pages * ATT_PAGE;
   const int qrow = cfg->d_nope + cfg->d_rope;
 
-  // (1) plan the split-KV work list on the device
+  // (1) Q̂ = [q_nope · W_UK | RoPE(q_rope)], one CTA per head and token tile (all 4 m-tiles of
+  //     d_c); one extra block plans the split-KV work list. Launched normally: the call's
+  //     inputs may come from the kernel just before it.
   mark(0);
-  PlanParams pp{seq_lens, batch, tq, L.n_mt, max_pos, L.P, L.max_segs,
-                L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
-  attn_plan_kernel<<<1, 1024, 0, st>>>(pp);
-
-  // (2) Q̂ = [q_nope · W_UK | RoPE(q_rope)]
-  mark(1);
   {
     CUtensorMap mA, mB;
     const uint64_t da[3] = {static_cast<uint64_t>(cfg->d_nope), ATT_DC, static_cast<uint64_t>(H)};
@@ -484,17 +536,23 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     const uint64_t db[3] = {static_cast<uint64_t>(qrow), static_cast<uint64_t>(H),
                             static_cast<uint64_t>(n_q)};
     const uint64_t sb[2] = {static_cast<uint64_t>(qrow) * 2, static_cast<uint64_t>(qrow) * 2 * H};
-    const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(pick_bn(n_q))};
+    // at most 128 tokens per CTA: 4 accumulators of bn columns fill TMEM's 512, and the ring
+    // plus the RoPE box stay within shared memory
+    const int bn = pick_bn(n_q) > 128 ? 128 : pick_bn(n_q);
+    const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(bn)};
     if (!make_map(&mA, w_uk_t, 3, da, sa, ba) || !make_map(&mB, q, 3, db, sb, bb))
       return MLA_ERR_CUDA;
-    GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1};
+    const int m_per_cta = ATT_DC / 128;
+    GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1, m_per_cta, 1};
+    PlanParams pp{seq_lens, batch, tq, L.n_mt, max_pos, L.P, L.max_segs,
+                  L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
     EpiQhat epi{L.qhat, static_cast<const __nv_bfloat16*>(q), seq_lens, H, tq, ATT_DC, ATT_DR,
-                cfg->d_nope, n_q, max_pos, cfg->rope_theta};
-    const mla_status s = launch_gemm(mA, mB, shp, ATT_DC / 128, H, epi, st);
+                cfg->d_nope, n_q, max_pos, bn, pp, rope_freqs(cfg)};
+    const mla_status s = launch_gemm(mA, mB, shp, ATT_DC / 128, H, epi, st, bn);
     if (s != MLA_OK) return s;
   }
 
-  // (3) fused latent attention, one partial per segment
+  // (2) fused latent attention, one partial per segment
   {
     CUtensorMap mc, mq;
     const uint64_t dc[2] = {ATT_ROW, static_cast<uint64_t>(num_pages) * ATT_PAGE};
@@ -509,38 +567,46 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
                   cfg->softmax_scale * 1.4426950408889634f};
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
-    mark(2);
-    mla_decode_attn_kernel<<<2 * L.P, ATT_THREADS, ATT_SMEM_BYTES, st>>>(mc, mq, ap);
-    const mla_status s = last_launch_status();
+    mark(1);
+    const mla_status s = launch_pdl(mla_decode_attn_kernel, dim3(2 * L.P), dim3(ATT_THREADS),
+                                    ATT_SMEM_BYTES, st, mc, mq, ap);
     if (s != MLA_OK) return s;
   }
 
-  // (4) merge split partials -> o_lat (bf16)
-  mark(3);
+  // (3) merge the split partials and project: out = o_lat · W_UVᵀ per head
   {
-    const int rows = batch * L.R;
-    attn_combine_kernel<<<(rows + 7) / 8, 256, 0, st>>>(L.o_part, L.lse, L.unit_seg, L.o_lat,
-                                                        rows, L.R, L.n_mt);
-    const mla_status s = last_launch_status();
-    if (s != MLA_OK) return s;
-  }
-
-  // (5) out = o_lat · W_UVᵀ per head
-  {
-    CUtensorMap mA, mB;
+    CUtensorMap mA;
     const uint64_t da[3] = {ATT_DC, static_cast<uint64_t>(cfg->d_v), static_cast<uint64_t>(H)};
     const uint64_t sa[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * cfg->d_v};
     const uint32_t ba[3] = {64, 128, 1};
-    const uint64_t db[3] = {ATT_DC, static_cast<uint64_t>(H), static_cast<uint64_t>(n_q)};
-    const uint64_t sb[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * H};
-    const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(pick_bn(n_q))};
-    if (!make_map(&mA, w_uv, 3, da, sa, ba) || !make_map(&mB, L.o_lat, 3, db, sb, bb))
-      return MLA_ERR_CUDA;
-    GemmShape shp{cfg->d_v, n_q, ATT_DC / 64, ATT_DC / 64, 1, 1};
-    EpiOut epi{static_cast<__nv_bfloat16*>(out), H, cfg->d_v};
-    mark(4);
-    const mla_status s = launch_gemm(mA, mB, shp, (cfg->d_v + 127) / 128, H, epi, st);
-    mark(5);
+    if (!make_map(&mA, w_uv, 3, da, sa, ba)) return MLA_ERR_CUDA;
+    VprojParams vp{L.o_part, L.lse, L.unit_seg, static_cast<__nv_bfloat16*>(out), H, tq, L.n_mt,
+                   n_q, cfg->d_v};
+    const int bn = pick_bn(n_q) > 64 ? 64 : pick_bn(n_q);
+    const dim3 grid((cfg->d_v + 127) / 128, (n_q + bn - 1) / bn, H);
+    mark(2);
+    mla_status s;
+    switch (bn) {
+      case 16:
+        s = allow_smem(vproj_merge_kernel<16>, vproj_smem_bytes<16>())
+                ? launch_pdl(vproj_merge_kernel<16>, grid, dim3(VP_THREADS),
+                             vproj_smem_bytes<16>(), st, mA, vp)
+                : MLA_ERR_CUDA;
+        break;
+      case 32:
+        s = allow_smem(vproj_merge_kernel<32>, vproj_smem_bytes<32>())
+                ? launch_pdl(vproj_merge_kernel<32>, grid, dim3(VP_THREADS),
+                             vproj_smem_bytes<32>(), st, mA, vp)
+                : MLA_ERR_CUDA;
+        break;
+      default:
+        s = allow_smem(vproj_merge_kernel<64>, vproj_smem_bytes<64>())
+                ? launch_pdl(vproj_merge_kernel<64>, grid, dim3(VP_THREADS),
+                             vproj_smem_bytes<64>(), st, mA, vp)
+                : MLA_ERR_CUDA;
+        break;
+    }
+    mark(3);
     return s;
   }
 }

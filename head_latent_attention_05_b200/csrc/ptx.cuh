@@ -99,6 +99,13 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t local_smem_addr, uint32
   return r;
 }
 
+// Load a float from the shared memory of another CTA of the cluster (address from map_to_rank).
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
 // Asynchronous 16-byte store into another CTA's shared memory; on completion it performs a
 // complete_tx of 16 bytes on the mbarrier at `remote_bar` (in that same CTA).
 __device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, uint32_t b,
@@ -221,6 +228,41 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
       : "memory");
 }
 
+// Warp-converged forms: every lane of a fully converged warp executes them and the one lane
+// that elect.sync picks (the same lane each time for the same converged warp) issues the MMA or
+// the commit. An issuing warp that stays converged like this issued N = 64 MMAs at ~37 cycles
+// each on B200 even with other warps busy; a single-lane, diverged issuer took 45-66.
+__device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                  uint64_t b_desc, uint32_t idesc,
+                                                  uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+__device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
+  asm volatile(
+      "{\n\t.reg .pred e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}\n" ::"r"(
+          smem_addr(bar))
+      : "memory");
+}
+
 // Warp-collective TMEM load: lane i of the warp reads TMEM lane (32*(warp%4) + i), 16 or 32
 // consecutive 32-bit columns starting at the column in taddr.
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
@@ -333,5 +375,17 @@ __device__ __forceinline__ float fast_exp2(float x) {
 }
 
 __device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31u) == 0u; }
+
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may
+// start while the previous kernel of the stream still runs; pdl_wait() blocks until that kernel
+// has completed and its writes are visible (a no-op for a normally launched kernel).
+// pdl_trigger() lets the next such kernel of the stream start early. The library's kernels
+// trigger only after their own pdl_wait() and after their TMEM allocation, so a kernel that has
+// started knows that every kernel two or more places before it in the stream has finished,
+// and a dependent CTA can never hold TMEM that a still-starting CTA of this grid waits for.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
 
 }  // namespace mla

@@ -7,6 +7,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace mla {
 
@@ -75,9 +76,11 @@ append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
                      const T* __restrict__ kv_gain, const int32_t* __restrict__ seq_idx,
                      const int32_t* __restrict__ pos, const int32_t* __restrict__ block_table,
                      int batch, int max_pages, T* __restrict__ cache, int num_pages,
-                     int page_size, int d_c, int d_r, float eps, float theta) {
+                     int page_size, int d_c, int d_r, float eps,
+                     const __grid_constant__ RopeFreqs rf) {
   __shared__ float red[32];
   extern __shared__ float row_s[];  // [d_c + d_r]
+  pdl_wait();   // the split-K partials of the GEMM just before are complete from here on
   const int i = blockIdx.x;
   const int row = d_c + d_r;
   const int b = seq_idx[i], p = pos[i];
@@ -91,8 +94,14 @@ append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
     const float* src = kv + static_cast<int64_t>(i) * row + f;
     const int64_t stride = static_cast<int64_t>(n_tok) * row;
     float v = 0.0f;
-#pragma unroll 8
-    for (int s = 0; s < n_splits; ++s) v += src[s * stride];
+    // 16 partials in flight per round, summed in split order
+    for (int s0 = 0; s0 < n_splits; s0 += 16) {
+      float part[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) part[j] = (s0 + j < n_splits) ? src[(s0 + j) * stride] : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v += part[j];
+    }
     row_s[f] = v;
     if (f < d_c) ss = fmaf(v, v, ss);
   }
@@ -102,9 +111,79 @@ append_finish_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
     dst[f] = Elem<T>::from_f(row_s[f] * rstd * Elem<T>::to_f(kv_gain[f]));
   for (int pr = threadIdx.x; pr < d_r / 2; pr += blockDim.x) {
     float ox, oy;
-    rope_pair(row_s[d_c + 2 * pr], row_s[d_c + 2 * pr + 1], pr, d_r, p, theta, &ox, &oy);
+    rope_pair(row_s[d_c + 2 * pr], row_s[d_c + 2 * pr + 1], rf.f_hi[pr], rf.f_lo[pr], p, &ox, &oy);
     dst[d_c + 2 * pr] = Elem<T>::from_f(ox);
     dst[d_c + 2 * pr + 1] = Elem<T>::from_f(oy);
+  }
+}
+
+// Cluster form of the same step, for the tensor-core append: the FIN_CLUSTER CTAs of a cluster
+// share one token (grid.x = FIN_CLUSTER * n_tok), each owning a contiguous, even-sized slice of
+// the row's features, so that the split-K partials are read by that many SMs at once (one SM
+// alone is limited by its outstanding misses, not by bandwidth). The RMSNorm's sum of squares
+// is combined over the cluster through distributed shared memory, in rank order, so the result
+// does not depend on timing. Every thread reaches both cluster barriers, whatever happens.
+constexpr int FIN_CLUSTER = 8;
+constexpr int FIN_THREADS = 128;
+
+template <typename T>
+__global__ void __launch_bounds__(FIN_THREADS)
+append_finish_cluster_kernel(const float* __restrict__ kv, int n_splits, int n_tok,
+                             const T* __restrict__ kv_gain, const int32_t* __restrict__ seq_idx,
+                             const int32_t* __restrict__ pos,
+                             const int32_t* __restrict__ block_table, int batch, int max_pages,
+                             T* __restrict__ cache, int num_pages, int page_size, int d_c,
+                             int d_r, float eps, const __grid_constant__ RopeFreqs rf) {
+  __shared__ float red[32];
+  __shared__ float ss_part;
+  extern __shared__ float slice_s[];   // this CTA's feature values
+  const int i = blockIdx.x / FIN_CLUSTER;
+  const uint32_t rank = cluster_ctarank();
+  const int row = d_c + d_r;
+  const int per = (((row + FIN_CLUSTER - 1) / FIN_CLUSTER) + 1) & ~1;   // even slice width
+  const int f0 = static_cast<int>(rank) * per, f1 = min(row, f0 + per);
+  // the destination comes from inputs of the call (complete before its first kernel ran):
+  // look it up while the GEMM still runs
+  const int b = seq_idx[i], p = pos[i];
+  T* dst = cache_row(cache, block_table, b, p, batch, max_pages, num_pages, page_size, row);
+  pdl_wait();   // the split-K partials of the GEMM just before are complete from here on
+  const int64_t stride = static_cast<int64_t>(n_tok) * row;
+  float ss = 0.0f;
+  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) {
+    const float* src = kv + static_cast<int64_t>(i) * row + f;
+    float v = 0.0f;
+    for (int s0 = 0; s0 < n_splits; s0 += 16) {   // 16 partials in flight, summed in order
+      float part[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) part[j] = (s0 + j < n_splits) ? src[(s0 + j) * stride] : 0.0f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) v += part[j];
+    }
+    slice_s[f - f0] = v;
+    if (f < d_c) ss = fmaf(v, v, ss);
+  }
+  ss = block_sum(ss, red);   // also orders the slice_s writes before the reads below
+  if (threadIdx.x == 0) ss_part = ss;
+  cluster_sync_all();
+  float total = 0.0f;
+  for (uint32_t r = 0; r < FIN_CLUSTER; ++r)
+    total += ld_shared_cluster_f32(map_to_rank(smem_addr(&ss_part), r));
+  cluster_sync_all();   // no CTA leaves while another may still read its ss_part
+  if (dst == nullptr) {
+    if (threadIdx.x == 0 && rank == 0) record_error(MLA_ERR_DEVICE_OOB);
+    return;
+  }
+  const float rstd = 1.0f / sqrtf(total / static_cast<float>(d_c) + eps);
+  for (int f = f0 + threadIdx.x; f < min(f1, d_c); f += blockDim.x)
+    dst[f] = Elem<T>::from_f(slice_s[f - f0] * rstd * Elem<T>::to_f(kv_gain[f]));
+  // rotary pairs (d_c + 2q, d_c + 2q + 1) never straddle a slice: d_c, f0 and per are even
+  const int r0 = max(f0, d_c);
+  for (int f = r0 + 2 * static_cast<int>(threadIdx.x); f < f1; f += 2 * blockDim.x) {
+    const int pr = (f - d_c) / 2;
+    float ox, oy;
+    rope_pair(slice_s[f - f0], slice_s[f + 1 - f0], rf.f_hi[pr], rf.f_lo[pr], p, &ox, &oy);
+    dst[f] = Elem<T>::from_f(ox);
+    dst[f + 1] = Elem<T>::from_f(oy);
   }
 }
 
@@ -119,7 +198,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 qabs_simt_kernel(const T* __restrict__ q, const T* __restrict__ w_uk_t,
                  const int32_t* __restrict__ seq_lens, float* __restrict__ qhat, int H, int Tq,
-                 int d_c, int d_r, int d_nope, int max_pos, float theta) {
+                 int d_c, int d_r, int d_nope, int max_pos,
+                 const __grid_constant__ RopeFreqs rf) {
   extern __shared__ float qs[];  // [d_nope + d_r]
   const int r = blockIdx.x;
   const int h = r % H, t = (r / H) % Tq, b = r / (H * Tq);
@@ -141,7 +221,7 @@ qabs_simt_kernel(const T* __restrict__ q, const T* __restrict__ w_uk_t,
   const int p = L - Tq + t;
   for (int pr = threadIdx.x; pr < d_r / 2; pr += blockDim.x) {
     float ox = 0.0f, oy = 0.0f;
-    if (ok) rope_pair(qs[d_nope + 2 * pr], qs[d_nope + 2 * pr + 1], pr, d_r, p, theta, &ox, &oy);
+    if (ok) rope_pair(qs[d_nope + 2 * pr], qs[d_nope + 2 * pr + 1], rf.f_hi[pr], rf.f_lo[pr], p, &ox, &oy);
     out[d_c + 2 * pr] = ox;
     out[d_c + 2 * pr + 1] = oy;
   }

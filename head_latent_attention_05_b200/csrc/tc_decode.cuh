@@ -2,10 +2,10 @@
 //
 // Work split. For sequence b the R = Tq*H query rows (row r = t*H + h) form ceil(R/128)
 // "units" of 128 rows; every unit attends over the sequence's pages (tiles of 64 tokens). A
-// planning kernel cuts the concatenated tile list of all units into P equal ranges, one per
-// pair of CTAs, so long and short sequences spread evenly over the GPU (split-KV). Each
-// range piece inside one unit is a "segment"; it produces a partial result (O / l, lse) that
-// the combine kernel merges by log-sum-exp.
+// planner (one extra block of the query-absorption GEMM) cuts the concatenated tile list of
+// all units into P equal ranges, one per pair of CTAs, so long and short sequences spread
+// evenly over the GPU (split-KV). Each range piece inside one unit is a "segment"; it produces
+// a partial result (O / l, lse) that the value-projection kernel merges by log-sum-exp.
 //
 // One pair of CTAs per range. Both CTAs run the same token tiles: each computes the full
 // score tile S = Q̂·Cᵀ (K = 576, heads on the MMA M side) and the same softmax, and accumulates
@@ -34,6 +34,7 @@
 // rescaled) when a new score exceeds it by more than 2^8, which keeps every P <= 256.
 #pragma once
 
+#include <climits>
 #include <type_traits>
 
 #include "common.cuh"
@@ -93,20 +94,28 @@ struct PlanParams {
   AttnSeg* segs;         // [max_segs]
 };
 
+constexpr int ATT_MAX_PAIRS = 1024;   // CTA pairs of the attention grid (one per two SMs)
+constexpr int ATT_SEG_COST_TILES = 5;  // planner's price of one more segment, in tiles
+
+// Start of pair p's tile range, p*T/P; the planner tabulates it once per call.
 __device__ __forceinline__ int64_t pair_start(int p, int64_t T, int P) {
   return (static_cast<int64_t>(p) * T) / P;
 }
-// Largest p in [0, P) with pair_start(p) <= x (x in [0, T)).
-__device__ __forceinline__ int pair_of(int64_t x, int64_t T, int P) {
-  int p = static_cast<int>((x * P) / T);
-  while (p + 1 < P && pair_start(p + 1, T, P) <= x) ++p;
-  while (p > 0 && pair_start(p, T, P) > x) --p;
-  return p;
+// Largest p in [0, P) with ps[p] <= x (x in [0, T)), by bisection over the table ps.
+__device__ __forceinline__ int pair_of(int64_t x, const int* ps, int P) {
+  int lo = 0, hi = P - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (ps[mid] <= x) lo = mid; else hi = mid - 1;
+  }
+  return lo;
 }
 
-// Block-wide exclusive scan of one int per thread (blockDim.x == 1024); returns the total.
+// Block-wide exclusive scan of one int per thread (blockDim.x a multiple of 32, at most 1024);
+// returns the total.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_tot) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n_warps = static_cast<int>(blockDim.x >> 5);
   int x = v;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -116,7 +125,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
   if (lane == 31) warp_tot[warp] = x;
   __syncthreads();
   if (warp == 0) {
-    int w = warp_tot[lane];
+    int w = lane < n_warps ? warp_tot[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int y = __shfl_up_sync(0xffffffffu, w, o);
@@ -127,19 +136,33 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
   __syncthreads();
   const int before = (warp > 0 ? warp_tot[warp - 1] : 0);
   *excl = before + x - v;
-  const int total = warp_tot[31];
+  const int total = warp_tot[n_warps - 1];
   __syncthreads();
   return total;
 }
 
-__global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
+// The planner, run by one whole block of any size (a multiple of 32): it rides along as an
+// extra block of the query-absorption GEMM, which runs just before the attention kernel.
+//
+// Balance. A CTA pair pays a fixed price each time it moves on to another unit (the finished
+// segment's epilogue and the next unit's Q̂ load lie on its critical path; measured at about
+// five tiles' worth on B200). So the tile list is cut in a virtual stream in which every unit
+// is followed by a gap of ATT_SEG_COST_TILES tiles: unit u occupies [vs_u, vs_u + n_u) with
+// vs_u = (tiles of units before u) + ATT_SEG_COST_TILES * u, and pair p takes the virtual range
+// [p*V/P, (p+1)*V/P). A pair whose range crosses into another unit then gets correspondingly
+// fewer tiles, and every pair carries about the same cost.
+__device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
   __shared__ int warp_tot[32];
   __shared__ int carry_s;
+  __shared__ int ps[ATT_MAX_PAIRS + 1];          // virtual start of pair p's range, p = 0..P
+  __shared__ int first_seg[ATT_MAX_PAIRS + 1];   // lowest segment index of each pair
+  constexpr int C = ATT_SEG_COST_TILES;
   const int U = pp.B * pp.n_mt;
-  // pass 1: tiles per unit -> global tile offsets
+  const int nt = static_cast<int>(blockDim.x);
+  // pass 1: tiles per unit -> virtual unit starts
   if (threadIdx.x == 0) carry_s = 0;
   __syncthreads();
-  for (int u0 = 0; u0 < U; u0 += 1024) {
+  for (int u0 = 0; u0 < U; u0 += nt) {
     const int u = u0 + threadIdx.x;
     int n = 0;
     if (u < U) {
@@ -153,28 +176,30 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
     }
     int excl;
     const int tot = block_exclusive_scan(n, &excl, warp_tot);
-    if (u < U) pp.unit_tiles[u] = carry_s + excl;
+    if (u < U) pp.unit_tiles[u] = carry_s + excl + C * u;
     __syncthreads();
     if (threadIdx.x == 0) carry_s += tot;
     __syncthreads();
   }
-  const int64_t T = carry_s;
+  const int V = carry_s + C * U;   // virtual length: all tiles and one gap per unit
+  for (int p = threadIdx.x; p <= pp.P; p += nt) {
+    ps[p] = static_cast<int>(pair_start(p, V, pp.P));
+    first_seg[p] = INT_MAX;
+  }
   __syncthreads();
-  // pass 2: segments per unit: one per pair whose (non-empty) tile range meets the unit's.
-  // When there are fewer tiles than pairs some pair ranges are empty; they get no segment.
+  // pass 2: segments per unit: one per pair whose range meets the unit's virtual range
   if (threadIdx.x == 0) carry_s = 0;
   __syncthreads();
-  for (int u0 = 0; u0 < U; u0 += 1024) {
+  for (int u0 = 0; u0 < U; u0 += nt) {
     const int u = u0 + threadIdx.x;
-    int nseg = 0, t0 = 0, t1 = 0, p0 = 0, p1 = -1;
+    int nseg = 0, v0 = 0, v1 = 0, p0 = 0, p1 = -1;
     if (u < U) {
-      t0 = pp.unit_tiles[u];
-      t1 = (u + 1 < U) ? pp.unit_tiles[u + 1] : static_cast<int>(T);
-      if (t1 > t0) {
-        p0 = pair_of(t0, T, pp.P);
-        p1 = pair_of(t1 - 1, T, pp.P);
-        for (int p = p0; p <= p1; ++p)
-          nseg += pair_start(p, T, pp.P) < pair_start(p + 1, T, pp.P) ? 1 : 0;
+      v0 = pp.unit_tiles[u];
+      v1 = ((u + 1 < U) ? pp.unit_tiles[u + 1] : V) - C;   // end of this unit's tiles
+      if (v1 > v0) {
+        p0 = pair_of(v0, ps, pp.P);
+        p1 = pair_of(v1 - 1, ps, pp.P);
+        for (int p = p0; p <= p1; ++p) nseg += min(v1, ps[p + 1]) > max(v0, ps[p]) ? 1 : 0;
       }
     }
     int excl;
@@ -184,15 +209,16 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
       pp.unit_seg[u] = s0;
       int i = 0;
       for (int p = p0; p <= p1; ++p) {
-        const int64_t a = max(static_cast<int64_t>(t0), pair_start(p, T, pp.P));
-        const int64_t e = min(static_cast<int64_t>(t1), pair_start(p + 1, T, pp.P));
+        const int a = max(v0, ps[p]);
+        const int e = min(v1, ps[p + 1]);
         if (e <= a) continue;
         AttnSeg sg;
         sg.unit = u;
-        sg.tile_begin = static_cast<int32_t>(a - t0);
-        sg.tile_end = static_cast<int32_t>(e - t0);
+        sg.tile_begin = a - v0;
+        sg.tile_end = e - v0;
         sg.pair = p;
         if (s0 + i < pp.max_segs) pp.segs[s0 + i] = sg;
+        atomicMin(&first_seg[p], s0 + i);
         ++i;
       }
     }
@@ -202,16 +228,12 @@ __global__ void __launch_bounds__(1024) attn_plan_kernel(PlanParams pp) {
   }
   const int S = carry_s;
   if (threadIdx.x == 0) pp.unit_seg[U] = S;
-  __syncthreads();
-  // pass 3: first segment of every pair (segments are ordered by pair)
-  for (int p = threadIdx.x; p <= pp.P; p += blockDim.x) {
-    // binary search: first segment whose pair >= p
-    int lo = 0, hi = S;
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if (pp.segs[mid].pair < p) lo = mid + 1; else hi = mid;
-    }
-    pp.pair_seg[p] = (p == pp.P) ? S : lo;
+  // pass 3: segments are ordered by pair; a pair without segments starts where the next pair
+  // that has some starts, and pair_seg[P] = S closes the list
+  for (int p = threadIdx.x; p <= pp.P; p += nt) {
+    int q = p;
+    while (q < pp.P && first_seg[q] == INT_MAX) ++q;
+    pp.pair_seg[p] = (q < pp.P) ? first_seg[q] : S;
   }
 }
 
@@ -289,12 +311,13 @@ __device__ __forceinline__ void att_qk_chunk(uint32_t tmem, uint64_t b_stage, ui
   for (int kk = 0; kk < 4; ++kk) {
     const uint32_t acc = (J == 0 && kk == 0) ? 0u : 1u;
     if constexpr (C < ATT_QT_ELEMS / 64)
-      mma_bf16_ts(tmem + TM_S, tmem + TM_Q + (C * 4 + kk) * 8, b0 + static_cast<uint64_t>(kk * 2),
-                  IDESC_QK, acc);
+      mma_bf16_ts_elect(tmem + TM_S, tmem + TM_Q + (C * 4 + kk) * 8,
+                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
     else
-      mma_bf16_ss(tmem + TM_S,
-                  qs_desc + static_cast<uint64_t>(((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES + kk * 32) >> 4),
-                  b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
+      mma_bf16_ss_elect(tmem + TM_S,
+                        qs_desc + static_cast<uint64_t>(
+                                      ((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES + kk * 32) >> 4),
+                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
   }
 }
 
@@ -311,7 +334,6 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;
-  const int seg_begin = p.pair_seg[pair], seg_end = p.pair_seg[pair + 1];
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ATT_STAGES; ++s) {
@@ -342,6 +364,9 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = sh.tmem_base;
+  pdl_wait();   // the plan and Q̂ of the previous kernel are complete and visible from here on
+  pdl_trigger();
+  const int seg_begin = p.pair_seg[pair], seg_end = p.pair_seg[pair + 1];
 
   if (seg_begin < seg_end) {
     if (warp == 0) {
@@ -389,6 +414,17 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           cp.next();
         };
         for (int i = 0; i < ATT_PREFETCH_AHEAD; ++i) prefetch_next();
+        // Q̂ rows of this pair's later segments into L2 now, so that switching units later
+        // reads them from L2 rather than HBM
+        if (half == 0) {
+          for (int s_i = seg_begin + 1; s_i < seg_end; ++s_i) {
+            const AttnSeg sg = p.segs[s_i];
+            const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
+            const int rows = min(128, p.R - mt * 128);
+            prefetch_l2_bulk(p.qhat + (static_cast<int64_t>(b) * p.R + mt * 128) * ATT_ROW,
+                             static_cast<uint32_t>(rows * ATT_ROW * 2));
+          }
+        }
         int gq = 0, go = 0;
         bool ok = true;
         load_q_smem(cq.sg);
@@ -428,19 +464,20 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           (void)mbar_wait(&sh.full_own[j % ATT_STAGES], (j / ATT_STAGES) & 1);
       }
     } else if (warp == 1) {
-      if (lane == 0) {
+      {
         // =========================================================== score MMA issuer
+        // (the whole warp runs this loop; one elected lane issues each MMA and commit)
         const uint32_t stage0 = smem_addr(stage_buf);
         const uint64_t qs_desc = smem_desc_sw128(smem_addr(qs_buf), 16, 1024);
         TileCursor cur;
         cur.init(p.segs, seg_begin, seg_end);
         for (int g = 0; cur.valid(); ++g, cur.next()) {
           const int st = g % ATT_STAGES;
-          if (cur.first_of_seg() && !att_wait(sh, &sh.q_full, cur.k & 1)) break;
-          if (g >= 1 && !att_wait(sh, &sh.s_free, (g - 1) & 1)) break;
+          if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) break;
+          if (g >= 1 && !att_warp_wait(sh, &sh.s_free, (g - 1) & 1)) break;
           const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
           // S over the score-only chunks first, then this CTA's own chunks (see att_chunk_order)
-          if (!att_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
+          if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
           if (half == 0) {
             att_qk_chunk<0, 0>(tmem, b_stage, qs_desc); att_qk_chunk<0, 1>(tmem, b_stage, qs_desc);
@@ -451,8 +488,8 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
             att_qk_chunk<1, 2>(tmem, b_stage, qs_desc); att_qk_chunk<1, 3>(tmem, b_stage, qs_desc);
             att_qk_chunk<1, 4>(tmem, b_stage, qs_desc);
           }
-          mma_commit(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
-          if (!att_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
+          mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
+          if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
           if (half == 0) {
             att_qk_chunk<0, 5>(tmem, b_stage, qs_desc); att_qk_chunk<0, 6>(tmem, b_stage, qs_desc);
@@ -461,16 +498,17 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
             att_qk_chunk<1, 5>(tmem, b_stage, qs_desc); att_qk_chunk<1, 6>(tmem, b_stage, qs_desc);
             att_qk_chunk<1, 7>(tmem, b_stage, qs_desc); att_qk_chunk<1, 8>(tmem, b_stage, qs_desc);
           }
-          mma_commit(&sh.s_full);
-          if (cur.last_of_seg()) mma_commit(&sh.q_free);
-          mma_commit(&sh.empty_own[st]);
+          mma_commit_elect(&sh.s_full);
+          if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
+          mma_commit_elect(&sh.empty_own[st]);
         }
         // drain: every MMA issued above completes before TMEM is released
-        mma_commit(&sh.drain);
-        (void)mbar_wait(&sh.drain, 0);
+        mma_commit_elect(&sh.drain);
+        if (lane == 0) (void)mbar_wait(&sh.drain, 0);
+        __syncwarp();
       }
     } else if (warp == 6) {
-      if (lane == 0) {
+      {   // the whole warp runs this loop; one elected lane issues
         // =========================================================== P·C MMA issuer
         constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
         const uint32_t stage0 = smem_addr(stage_buf);
@@ -480,21 +518,22 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         for (int g = 0; cur.valid(); ++g, cur.next()) {
           const int st = g % ATT_STAGES;
           const bool first = cur.first_of_seg();
-          if (first && cur.k >= 1 && !att_wait(sh, &sh.o_free, (cur.k - 1) & 1)) break;
-          if (!att_wait(sh, &sh.p_full, g & 1)) break;
+          if (first && cur.k >= 1 && !att_warp_wait(sh, &sh.o_free, (cur.k - 1) & 1)) break;
+          if (!att_warp_wait(sh, &sh.p_full, g & 1)) break;
           tc_fence_after_sync();
           // O_half += P · C[:, own half]: chunks 4*half .. 4*half+3, read MN-major (N = 256)
           const uint64_t b0 = smem_desc_sw128(
               stage0 + st * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES, ATT_CHUNK_BYTES, 1024);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 16 tokens per K-step
-            mma_bf16_ss(tmem + TM_O, p_desc + static_cast<uint64_t>(kk * 2),
+            mma_bf16_ss_elect(tmem + TM_O, p_desc + static_cast<uint64_t>(kk * 2),
                         b0 + static_cast<uint64_t>(kk * 128), IDESC_PV, (first && kk == 0) ? 0u : 1u);
-          mma_commit(&sh.empty_own[st]);
-          mma_commit(&sh.pv_done);
+          mma_commit_elect(&sh.empty_own[st]);
+          mma_commit_elect(&sh.pv_done);
         }
-        mma_commit(&sh.drain);
-        (void)mbar_wait(&sh.drain, 0);
+        mma_commit_elect(&sh.drain);
+        if (lane == 0) (void)mbar_wait(&sh.drain, 0);
+        __syncwarp();
       }
     } else {
       // ============================================================ softmax warps
@@ -694,49 +733,6 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
     __syncwarp();
     tc_fence_after_sync();
     tmem_dealloc(tmem, 512);
-  }
-}
-
-// ------------------------------------------------------------------------ split-KV combine
-// One warp per query row g = b*R + r: merge the row's partials (one per segment of its unit)
-// by their base-2 log-sum-exp and store o_lat in bf16 (the B operand of the value projection).
-__global__ void __launch_bounds__(256)
-attn_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ lse,
-                    const int32_t* __restrict__ unit_seg, __nv_bfloat16* __restrict__ o_lat,
-                    int n_rows, int R, int n_mt) {
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int gr = blockIdx.x * 8 + warp;
-  if (gr >= n_rows) return;
-  const int b = gr / R, r = gr % R;
-  const int u = b * n_mt + r / 128, rl = r % 128;
-  const int s0 = unit_seg[u], s1 = unit_seg[u + 1];
-  float mx = -INFINITY;
-  for (int s = s0; s < s1; ++s) mx = fmaxf(mx, lse[static_cast<int64_t>(s) * 128 + rl]);
-  float4 acc[4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float den = 0.0f;
-  if (mx > -INFINITY) {
-    for (int s = s0; s < s1; ++s) {
-      const float w = exp2f(lse[static_cast<int64_t>(s) * 128 + rl] - mx);
-      den += w;
-      const float4* src = reinterpret_cast<const float4*>(o_part + (static_cast<int64_t>(s) * 128 + rl) * ATT_DC);
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 v = src[lane + 32 * i];
-        acc[i].x = fmaf(w, v.x, acc[i].x);
-        acc[i].y = fmaf(w, v.y, acc[i].y);
-        acc[i].z = fmaf(w, v.z, acc[i].z);
-        acc[i].w = fmaf(w, v.w, acc[i].w);
-      }
-    }
-  }
-  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-  uint2* dst = reinterpret_cast<uint2*>(o_lat + static_cast<int64_t>(gr) * ATT_DC);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    dst[lane + 32 * i] = make_uint2(pack_bf16x2(acc[i].x * inv, acc[i].y * inv),
-                                    pack_bf16x2(acc[i].z * inv, acc[i].w * inv));
   }
 }
 

@@ -59,6 +59,7 @@ typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1 } mla_dtype;
  * rope_theta is the RoPE base: pair i of a d_rope-wide vector at position p turns by
  * p * rope_theta^(-2i/d_rope) (「淺析DeepSeek多頭潛在注意力機制（MLA）」, "MLA與ROPE的融合";
  * pairs are adjacent elements (2i, 2i+1)). page_size is the number of tokens per cache page.
+ * Every entry point rejects d_rope > 128 with MLA_ERR_UNSUPPORTED.
  */
 typedef struct {
   int32_t n_heads;
@@ -150,13 +151,15 @@ mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32
 
 /*
  * mla_decode with per-kernel timing: identical arguments and results, plus `events`, an array
- * of 6 cudaEvent_t created by the caller. events[i] is recorded on `stream` just before decode
- * kernel i (0 planning, 1 query absorption, 2 latent attention, 3 split combine, 4 value
- * projection) and events[5] after the last one, so cudaEventElapsedTime(events[2], events[3])
- * is the attention kernel's device time. While `stream` is being captured the events are
- * recorded with cudaEventRecordExternal, so they become event-record nodes of the graph. On the fp32 path, which
- * has no planning or combine kernel, events 0/1 mark the start and 3/4 the end of attention.
- * NULL entries are skipped.
+ * of 4 cudaEvent_t created by the caller, recorded on `stream` at the kernel boundaries of the
+ * bf16 path: events[0] before the query absorption (whose extra block also plans the split-KV
+ * work), events[1] before the latent attention kernel, events[2] before the fused split merge
+ * + value projection, events[3] after it; cudaEventElapsedTime(events[1], events[2]) is the
+ * attention kernel's device time. The event records sit between the kernels, so kernels that
+ * otherwise overlap their start with the previous kernel's end (programmatic dependent launch)
+ * run back to back here. While `stream` is being captured the events are recorded with
+ * cudaEventRecordExternal, so they become event-record nodes of the graph. The fp32 path marks
+ * the same three stages (absorption, attention, projection). NULL entries are skipped.
  */
 mla_status mla_decode_profiled(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
                                const void* cache, int32_t num_pages, const int32_t* block_table,
