@@ -265,7 +265,8 @@ struct DecodeLayout {
   int32_t *unit_tiles, *unit_seg, *pair_seg;
   AttnSeg* segs;
   __nv_bfloat16* qhat;
-  float *o_part, *lse;
+  __nv_bfloat16* o_part;
+  float* lse;
   size_t bytes;
 };
 
@@ -290,7 +291,7 @@ DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
   L.pair_seg = cv.take<int32_t>(L.P + 1);
   L.segs = cv.take<AttnSeg>(L.max_segs);
   L.qhat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_ROW);
-  L.o_part = cv.take<float>(static_cast<size_t>(L.max_segs) * 128 * ATT_DC);
+  L.o_part = cv.take<__nv_bfloat16>(static_cast<size_t>(L.max_segs) * 128 * ATT_DC);
   L.lse = cv.take<float>(static_cast<size_t>(L.max_segs) * 128);
   L.bytes = cv.off;
   return L;

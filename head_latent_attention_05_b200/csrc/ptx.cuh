@@ -137,6 +137,27 @@ __device__ __forceinline__ void cluster_sync_all() {
       "barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 
+// L2 cache policy that keeps the lines it is attached to over evict-normal ones (for data a
+// later kernel reads back soon, while a long stream passes through L2).
+__device__ __forceinline__ uint64_t l2_policy_evict_last() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+__device__ __forceinline__ void st_global_v4_hint(float* dst, float a, float b, float c, float d,
+                                                  uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "f"(a),
+               "f"(b), "f"(c), "f"(d), "l"(pol)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_global_u4_hint(void* dst, uint32_t a, uint32_t b, uint32_t c,
+                                                  uint32_t d, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(a),
+               "r"(b), "r"(c), "r"(d), "l"(pol)
+               : "memory");
+}
+
 // Make generic-proxy shared-memory writes visible to the async proxy (TMA, tcgen05.mma).
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

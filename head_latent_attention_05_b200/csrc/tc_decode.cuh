@@ -76,7 +76,7 @@ struct AttnParams {
   const int32_t* pair_seg;   // [P + 1]: pair p runs segments [pair_seg[p], pair_seg[p+1])
   const __nv_bfloat16* qhat; // [B*R][576]
   const __nv_bfloat16* cache;  // [num_pages][64][576] (for L2 prefetch)
-  float* o_part;             // [max_segs][128][512]
+  __nv_bfloat16* o_part;     // [max_segs][128][512] per-segment O / l, rounded to bf16
   float* lse;                // [max_segs][128]   (base-2 log-sum-exp of the scaled scores)
   int max_pages, num_pages;
   int H, Tq, R, n_mt;
@@ -705,17 +705,24 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         if (!att_warp_wait(sh, &sh.pv_done, seg_last_g & 1)) { ok = false; break; }
         tc_fence_after_sync();
         const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
-        float* dst = p.o_part + (static_cast<int64_t>(s_i) * 128 + r_local) * ATT_DC + half * 256;
+        __nv_bfloat16* dst =
+            p.o_part + (static_cast<int64_t>(s_i) * 128 + r_local) * ATT_DC + half * 256;
+        // the merge reads these partials right after this kernel: keep them in L2 while the
+        // cache stream of the other CTAs passes through it
+        const uint64_t keep = l2_policy_evict_last();
 #pragma unroll 1
         for (int c0 = hc * 128; c0 < hc * 128 + 128; c0 += 32) {
           uint32_t o[32];
           tmem_ld32(tmem + t_lane + TM_O + c0, o);
           tmem_ld_wait();
 #pragma unroll
-          for (int j = 0; j < 32; j += 4)
-            *reinterpret_cast<float4*>(dst + c0 + j) =
-                make_float4(__uint_as_float(o[j]) * inv_l, __uint_as_float(o[j + 1]) * inv_l,
-                            __uint_as_float(o[j + 2]) * inv_l, __uint_as_float(o[j + 3]) * inv_l);
+          for (int j = 0; j < 32; j += 8)
+            st_global_u4_hint(dst + c0 + j,
+                              pack_bf16x2(__uint_as_float(o[j]) * inv_l, __uint_as_float(o[j + 1]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[j + 2]) * inv_l, __uint_as_float(o[j + 3]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[j + 4]) * inv_l, __uint_as_float(o[j + 5]) * inv_l),
+                              pack_bf16x2(__uint_as_float(o[j + 6]) * inv_l, __uint_as_float(o[j + 7]) * inv_l),
+                              keep);
         }
         if (half == 0 && hc == 0)
           p.lse[static_cast<int64_t>(s_i) * 128 + r_local] =

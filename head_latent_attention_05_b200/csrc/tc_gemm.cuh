@@ -202,7 +202,7 @@ struct EpiSplitK {
   float* partial;
   int n_tok, F;
   struct SideState {};
-  static constexpr int side_bytes(int) { return 0; }
+  __host__ __device__ static constexpr int side_bytes(int) { return 0; }
   __device__ void aux() const {}
   __device__ SideState side_begin(int, int, int) const { return {}; }
   __device__ void side_issue(const CUtensorMap*, uint8_t*, uint64_t*, int, int) const {}
@@ -232,7 +232,7 @@ struct EpiQhat {
   struct SideState {
     int len;   // seq_lens of the first token this thread handles
   };
-  static constexpr int side_bytes(int bn) { return bn * 128; }
+  __host__ __device__ static constexpr int side_bytes(int bn) { return bn * 128; }
   __device__ bool rope_cta() const { return blockIdx.x == 0; }
   __device__ SideState side_begin(int tid, int nt, int n0) const {
     SideState st{-1};

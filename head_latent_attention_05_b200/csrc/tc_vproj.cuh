@@ -16,7 +16,7 @@
 namespace mla {
 
 struct VprojParams {
-  const float* o_part;        // [segments][128][512] per-segment O / l (fp32)
+  const __nv_bfloat16* o_part;  // [segments][128][512] per-segment O / l (bf16)
   const float* lse;           // [segments][128] base-2 log-sum-exp of each partial
   const int32_t* unit_seg;    // [U + 1] first segment of each unit
   __nv_bfloat16* out;         // [n_q][H][d_v]
@@ -71,8 +71,9 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
   __syncthreads();
   tc_fence_after_sync();
   const uint32_t tmem = tmem_base_s;
-  // ---- merge. 16 threads per B row, 16 rows per pass; thread k of a row owns the float4
-  // groups k + 16 i (i = 0..7) of the row's 512 dims, i.e. 16-byte piece k/2 of K-chunk i.
+  // ---- merge. 16 threads per B row, 16 rows per pass; thread k of a row owns the 16-byte
+  // groups q = k + 16 i (i = 0..3) of the row's 512 bf16 dims, i.e. 16-byte piece k%8 of
+  // K-chunk 2i + k/8.
   constexpr int RP = 16, TPR = VP_THREADS / RP, PASSES = BN / RP;
   const int rr_l = threadIdx.x / TPR, k = threadIdx.x % TPR;
   // the segment lists were written two kernels back (by the planner): read them before waiting
@@ -101,39 +102,39 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
 #pragma unroll
     for (int o = TPR / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float den = 0.0f;
-    float4 acc[8];
+    float acc[32];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
     if (mx > -INFINITY) {
       for (int s = s0 + k; s < s1; s += TPR) den += exp2f(p.lse[static_cast<int64_t>(s) * 128 + rl] - mx);
-      // two segments' loads in flight at a time; the sum runs in segment order
-      for (int sb = s0; sb < s1; sb += 2) {
-        const bool two = sb + 1 < s1;
-        const float w0 = exp2f(p.lse[static_cast<int64_t>(sb) * 128 + rl] - mx);
-        const float w1 = two ? exp2f(p.lse[static_cast<int64_t>(sb + 1) * 128 + rl] - mx) : 0.0f;
-        const float4* src0 = reinterpret_cast<const float4*>(
-            p.o_part + (static_cast<int64_t>(sb) * 128 + rl) * ATT_DC);
-        const float4* src1 = src0 + ATT_DC / 4 * 128;   // segment sb + 1, same row
-        float4 v0[8], v1[8];
+      // four segments' loads in flight at a time; the sum runs in segment order
+      for (int sb = s0; sb < s1; sb += 4) {
+        float w[4];
+        uint4 v[4][4];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          v0[i] = src0[k + TPR * i];
-          v1[i] = two ? src1[k + TPR * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 4; ++j) {
+          const int s = sb + j;
+          w[j] = 0.0f;
+          if (s < s1) {
+            w[j] = exp2f(p.lse[static_cast<int64_t>(s) * 128 + rl] - mx);
+            const uint4* src = reinterpret_cast<const uint4*>(
+                p.o_part + (static_cast<int64_t>(s) * 128 + rl) * ATT_DC);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) v[j][i] = src[k + TPR * i];
+          }
         }
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          acc[i].x = fmaf(w0, v0[i].x, acc[i].x);
-          acc[i].y = fmaf(w0, v0[i].y, acc[i].y);
-          acc[i].z = fmaf(w0, v0[i].z, acc[i].z);
-          acc[i].w = fmaf(w0, v0[i].w, acc[i].w);
-        }
-        if (two) {
+        for (int j = 0; j < 4; ++j) {
+          if (sb + j >= s1) break;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            acc[i].x = fmaf(w1, v1[i].x, acc[i].x);
-            acc[i].y = fmaf(w1, v1[i].y, acc[i].y);
-            acc[i].z = fmaf(w1, v1[i].z, acc[i].z);
-            acc[i].w = fmaf(w1, v1[i].w, acc[i].w);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t u[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+              acc[8 * i + 2 * e] = fmaf(w[j], f.x, acc[8 * i + 2 * e]);
+              acc[8 * i + 2 * e + 1] = fmaf(w[j], f.y, acc[8 * i + 2 * e + 1]);
+            }
           }
         }
       }
@@ -141,12 +142,15 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
 #pragma unroll
     for (int o = TPR / 2; o > 0; o >>= 1) den += __shfl_xor_sync(0xffffffffu, den, o);
     const float inv = den > 0.0f ? 1.0f / den : 0.0f;
-    // dims 4*(k + 16 i) .. +3: K-chunk i, 16-byte piece k/2, 8-byte half k%2 (swizzled row rr)
+    // group q = k + 16 i: K-chunk 2i + k/8, 16-byte piece k%8 of row rr (swizzled)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      uint8_t* dst = b_buf + i * B_CHUNK + rr * 128 + (((k >> 1) ^ (rr & 7)) << 4) + ((k & 1) << 3);
-      *reinterpret_cast<uint2*>(dst) = make_uint2(pack_bf16x2(acc[i].x * inv, acc[i].y * inv),
-                                                  pack_bf16x2(acc[i].z * inv, acc[i].w * inv));
+    for (int i = 0; i < 4; ++i) {
+      uint8_t* dst = b_buf + (2 * i + (k >> 3)) * B_CHUNK + rr * 128 + (((k & 7) ^ (rr & 7)) << 4);
+      *reinterpret_cast<uint4*>(dst) = make_uint4(
+          pack_bf16x2(acc[8 * i + 0] * inv, acc[8 * i + 1] * inv),
+          pack_bf16x2(acc[8 * i + 2] * inv, acc[8 * i + 3] * inv),
+          pack_bf16x2(acc[8 * i + 4] * inv, acc[8 * i + 5] * inv),
+          pack_bf16x2(acc[8 * i + 6] * inv, acc[8 * i + 7] * inv));
     }
   }
   fence_proxy_async_smem();

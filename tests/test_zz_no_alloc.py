@@ -45,10 +45,12 @@ def test_noalloc_decode_matches_decode_on_consecutive_calls():
 
 def test_noalloc_rejects_a_batch_beyond_its_scratch():
     cfg = Hs.config_of(V2)
-    assert mla.mla_decode_workspace_size(cfg, 64, 1) > mla.MLA_DECODE_NOALLOC_MAX_SCRATCH
+    big = 64   # the smallest power-of-two batch whose scratch exceeds the built-in array
+    while mla.mla_decode_workspace_size(cfg, big, 1) <= mla.MLA_DECODE_NOALLOC_MAX_SCRATCH:
+        big *= 2
     c = Hs.make_case(W.small_variant(V2, B=2), torch.tensor([64, 64], dtype=torch.int32))
-    q = torch.zeros((64, 1, V2.H, V2.d_nope + V2.d_r), dtype=torch.bfloat16, device="cuda")
-    out = torch.empty((64, 1, V2.H, V2.d_v), dtype=torch.bfloat16, device="cuda")
+    q = torch.zeros((big, 1, V2.H, V2.d_nope + V2.d_r), dtype=torch.bfloat16, device="cuda")
+    out = torch.empty((big, 1, V2.H, V2.d_v), dtype=torch.bfloat16, device="cuda")
     with pytest.raises(mla.MlaError) as e:
         mla.mla_decode_noalloc(cfg, q, c.d["cache"], c.d["block_table"], c.d["seq_lens"],
                                c.d["w_uk_t"], c.d["w_uv"], out)
