@@ -464,11 +464,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
 
 def kernel_sha() -> str:
-    """Hash of the attention kernel source, to tell whether stored counters are current."""
+    """Hash of the attention kernel's code (its source with // comments and blank lines
+    dropped), to tell whether stored counters are still current."""
     import hashlib
+    import re
     path = os.path.join(ROOT, "head_latent_attention_05_b200", "csrc", "tc_decode.cuh")
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    with open(path, encoding="utf-8") as f:
+        lines = [re.sub(r"//.*", "", ln).rstrip() for ln in f]
+    code = "\n".join(ln for ln in lines if ln.strip())
+    return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 
 def main():

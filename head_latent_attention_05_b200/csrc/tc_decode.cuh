@@ -24,8 +24,9 @@
 // score MMA consumes the early chunks first, so the late chunks' load latency hides behind it.
 //
 // Warp roles (352 threads): warp 0 TMA producer, warp 1 issues the score MMAs, warp 6 issues
-// the P·C MMAs (a single thread issues at most one tcgen05.mma per ~48 cycles, so the two
-// streams get their own threads; each accumulator still has a single issuer, which keeps the
+// the P·C MMAs (the two streams get their own warps; each warp stays converged and issues
+// through elect.sync, which on B200 keeps the issue rate at ~37 cycles per N = 64 MMA even
+// while the softmax warps are busy; each accumulator has a single issuer, which keeps the
 // summation order, and the result, deterministic). Warps 2..5 and 7..10 run the softmax,
 // rescale and epilogue: warp w owns TMEM lanes 32*(w%4).. (query rows), and the two warps of a
 // lane quarter split each row's 64 scores (columns 0..31 and 32..63), agreeing on the row
