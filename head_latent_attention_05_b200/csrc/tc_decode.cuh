@@ -301,24 +301,31 @@ __device__ __forceinline__ int att_chunk_order(int half, int j) {
   return j < 4 ? 4 * (1 - half) + j : (j == 4 ? 8 : 4 * half + (j - 5));
 }
 
-// Four K = 16 steps of S over chunk C = att_chunk_order(HALF, J) of a stage: A = Q̂[:, 64C ..
-// 64C+63] (TMEM for C < 6, the smem part above), B = the stage's chunk C. J == 0 overwrites S.
-template <int HALF, int J>
-__device__ __forceinline__ void att_qk_chunk(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc) {
+// Score K-steps of chunks j0..j1-1 (in att_chunk_order) of one tile: A = Q̂[:, 64C .. 64C+63]
+// (TMEM for C < 6, the smem part above), B = the stage's chunk C; the tile's first K-step
+// overwrites S. A compact loop (4 MMAs unrolled per chunk) rather than 36 unrolled MMAs: the
+// issuing warp shares the SM's instruction cache with the producer, P·C and softmax code.
+__device__ __forceinline__ void att_qk_part(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
+                                            int half, int j0, int j1) {
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
-  constexpr int C = J < 4 ? 4 * (1 - HALF) + J : (J == 4 ? 8 : 4 * HALF + (J - 5));
-  const uint64_t b0 = b_stage + static_cast<uint64_t>((C * ATT_CHUNK_BYTES) >> 4);
+#pragma unroll 1
+  for (int j = j0; j < j1; ++j) {
+    const int C = att_chunk_order(half, j);
+    const uint64_t b0 = b_stage + static_cast<uint64_t>((C * ATT_CHUNK_BYTES) >> 4);
+    if (C < ATT_QT_ELEMS / 64) {
+      const uint32_t a0 = tmem + TM_Q + C * 32;
 #pragma unroll
-  for (int kk = 0; kk < 4; ++kk) {
-    const uint32_t acc = (J == 0 && kk == 0) ? 0u : 1u;
-    if constexpr (C < ATT_QT_ELEMS / 64)
-      mma_bf16_ts_elect(tmem + TM_S, tmem + TM_Q + (C * 4 + kk) * 8,
-                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
-    else
-      mma_bf16_ss_elect(tmem + TM_S,
-                        qs_desc + static_cast<uint64_t>(
-                                      ((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES + kk * 32) >> 4),
-                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, acc);
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ts_elect(tmem + TM_S, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
+                          (j == 0 && kk == 0) ? 0u : 1u);
+    } else {
+      const uint64_t a0 =
+          qs_desc + static_cast<uint64_t>(((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES) >> 4);
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_bf16_ss_elect(tmem + TM_S, a0 + static_cast<uint64_t>(kk * 2),
+                          b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, 1u);
+    }
   }
 }
 
@@ -480,25 +487,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           // S over the score-only chunks first, then this CTA's own chunks (see att_chunk_order)
           if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          if (half == 0) {
-            att_qk_chunk<0, 0>(tmem, b_stage, qs_desc); att_qk_chunk<0, 1>(tmem, b_stage, qs_desc);
-            att_qk_chunk<0, 2>(tmem, b_stage, qs_desc); att_qk_chunk<0, 3>(tmem, b_stage, qs_desc);
-            att_qk_chunk<0, 4>(tmem, b_stage, qs_desc);
-          } else {
-            att_qk_chunk<1, 0>(tmem, b_stage, qs_desc); att_qk_chunk<1, 1>(tmem, b_stage, qs_desc);
-            att_qk_chunk<1, 2>(tmem, b_stage, qs_desc); att_qk_chunk<1, 3>(tmem, b_stage, qs_desc);
-            att_qk_chunk<1, 4>(tmem, b_stage, qs_desc);
-          }
+          att_qk_part(tmem, b_stage, qs_desc, half, 0, 5);
           mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
           if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          if (half == 0) {
-            att_qk_chunk<0, 5>(tmem, b_stage, qs_desc); att_qk_chunk<0, 6>(tmem, b_stage, qs_desc);
-            att_qk_chunk<0, 7>(tmem, b_stage, qs_desc); att_qk_chunk<0, 8>(tmem, b_stage, qs_desc);
-          } else {
-            att_qk_chunk<1, 5>(tmem, b_stage, qs_desc); att_qk_chunk<1, 6>(tmem, b_stage, qs_desc);
-            att_qk_chunk<1, 7>(tmem, b_stage, qs_desc); att_qk_chunk<1, 8>(tmem, b_stage, qs_desc);
-          }
+          att_qk_part(tmem, b_stage, qs_desc, half, 5, 9);
           mma_commit_elect(&sh.s_full);
           if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
           mma_commit_elect(&sh.empty_own[st]);
