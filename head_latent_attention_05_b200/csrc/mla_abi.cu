@@ -555,13 +555,18 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
 
   // (2) fused latent attention, one partial per segment
   {
-    CUtensorMap mc, mq;
+    CUtensorMap mc, mc4, mq;
     const uint64_t dc[2] = {ATT_ROW, static_cast<uint64_t>(num_pages) * ATT_PAGE};
     const uint64_t sc[1] = {ATT_ROW * 2};
     const uint32_t bc[2] = {64, ATT_PAGE};
+    // the same cache as [chunk of 64 dims][token][64 dims], 4 chunks of one page per box
+    const uint64_t dc4[3] = {64, static_cast<uint64_t>(num_pages) * ATT_PAGE, ATT_ROW / 64};
+    const uint64_t sc4[2] = {ATT_ROW * 2, 128};
+    const uint32_t bc4[3] = {64, ATT_PAGE, 4};
     const uint64_t dq[2] = {ATT_ROW, static_cast<uint64_t>(batch) * L.R};
     const uint32_t bq[2] = {64, 128};
-    if (!make_map(&mc, cache, 2, dc, sc, bc) || !make_map(&mq, L.qhat, 2, dq, sc, bq))
+    if (!make_map(&mc, cache, 2, dc, sc, bc) || !make_map(&mc4, cache, 3, dc4, sc4, bc4) ||
+        !make_map(&mq, L.qhat, 2, dq, sc, bq))
       return MLA_ERR_CUDA;
     AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat,
                   static_cast<const __nv_bfloat16*>(cache), L.o_part, L.lse,
@@ -570,7 +575,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
     mark(1);
     const mla_status s = launch_pdl(mla_decode_attn_kernel, dim3(2 * L.P), dim3(ATT_THREADS),
-                                    ATT_SMEM_BYTES, st, mc, mq, ap);
+                                    ATT_SMEM_BYTES, st, mc, mc4, mq, ap);
     if (s != MLA_OK) return s;
   }
 

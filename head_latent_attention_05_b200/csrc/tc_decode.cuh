@@ -331,6 +331,7 @@ __device__ __forceinline__ void att_qk_part(uint32_t tmem, uint64_t b_stage, uin
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
+                       const __grid_constant__ CUtensorMap map_cache4,
                        const __grid_constant__ CUtensorMap map_qhat, AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -362,6 +363,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
     sh.abort_flag = 0;
     fence_mbar_init();
     tma_prefetch_desc(&map_cache);
+    tma_prefetch_desc(&map_cache4);
     tma_prefetch_desc(&map_qhat);
   }
   if (warp == 1) {
@@ -391,15 +393,16 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           }
           return page;
         };
+        // A page's chunks c..c+3 come in one box of the 3-D view [chunk][token][64 dims] (TMA
+        // instructions are slow to issue, so fewer, larger boxes), the rope chunk 8 in its own.
         auto load_chunks = [&](const TileCursor& c, int g, bool own, uint64_t* bar) {
           const int page = page_of(c);
           uint8_t* st = stage_buf + (g % ATT_STAGES) * ATT_TILE_BYTES;
+          const int c0 = own ? 4 * half : 4 * (1 - half);
           mbar_arrive_expect_tx(bar, (own ? 4 : 5) * ATT_CHUNK_BYTES);
-          for (int j = own ? 5 : 0; j < (own ? 9 : 5); ++j) {
-            const int c_idx = att_chunk_order(half, j);
-            tma_load_2d(st + c_idx * ATT_CHUNK_BYTES, &map_cache, bar, 64 * c_idx,
-                        page * ATT_PAGE);
-          }
+          tma_load_3d(st + c0 * ATT_CHUNK_BYTES, &map_cache4, bar, 0, page * ATT_PAGE, c0);
+          if (!own)
+            tma_load_2d(st + 8 * ATT_CHUNK_BYTES, &map_cache, bar, 64 * 8, page * ATT_PAGE);
         };
         auto load_q_smem = [&](const AttnSeg& sg) {   // Q̂[:, 384:576] of a unit
           const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
