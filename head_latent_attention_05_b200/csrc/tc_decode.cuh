@@ -301,31 +301,58 @@ __device__ __forceinline__ int att_chunk_order(int half, int j) {
   return j < 4 ? 4 * (1 - half) + j : (j == 4 ? 8 : 4 * half + (j - 5));
 }
 
-// Score K-steps of chunks j0..j1-1 (in att_chunk_order) of one tile: A = Q̂[:, 64C .. 64C+63]
-// (TMEM for C < 6, the smem part above), B = the stage's chunk C; the tile's first K-step
-// overwrites S. A compact loop (4 MMAs unrolled per chunk) rather than 36 unrolled MMAs: the
-// issuing warp shares the SM's instruction cache with the producer, P·C and softmax code.
-__device__ __forceinline__ void att_qk_part(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
-                                            int half, int j0, int j1) {
+// Score K-steps over a run of consecutive chunks c .. c+n-1 of a tile. In the A-from-TMEM form
+// (chunks below 6: Q̂[:, 0:384] sits in TMEM) and the A-from-smem form (Q̂[:, 384:576]). Each
+// run is a short loop whose descriptors only step by constants: the issuing warp shares the
+// instruction cache with the producer, P·C and softmax code (a fully unrolled tile costs more
+// overall), and per-chunk index arithmetic or branching measured ~20 cycles per MMA.
+__device__ __forceinline__ void att_qk_ts(uint32_t tmem, uint64_t b_stage, int c, int n,
+                                          bool first) {
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
+  uint64_t b0 = b_stage + static_cast<uint64_t>((c * ATT_CHUNK_BYTES) >> 4);
+  uint32_t a0 = tmem + TM_Q + c * 32;
 #pragma unroll 1
-  for (int j = j0; j < j1; ++j) {
-    const int C = att_chunk_order(half, j);
-    const uint64_t b0 = b_stage + static_cast<uint64_t>((C * ATT_CHUNK_BYTES) >> 4);
-    if (C < ATT_QT_ELEMS / 64) {
-      const uint32_t a0 = tmem + TM_Q + C * 32;
+  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += 32) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ts_elect(tmem + TM_S, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
-                          (j == 0 && kk == 0) ? 0u : 1u);
-    } else {
-      const uint64_t a0 =
-          qs_desc + static_cast<uint64_t>(((C - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES) >> 4);
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16_ts_elect(tmem + TM_S, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
+                        (first && i == 0 && kk == 0) ? 0u : 1u);
+  }
+}
+__device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
+                                          int c, int n) {
+  constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
+  uint64_t b0 = b_stage + static_cast<uint64_t>((c * ATT_CHUNK_BYTES) >> 4);
+  uint64_t a0 =
+      qs_desc + static_cast<uint64_t>(((c - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES) >> 4);
+#pragma unroll 1
+  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += ATT_QS_CHUNK_BYTES >> 4) {
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_bf16_ss_elect(tmem + TM_S, a0 + static_cast<uint64_t>(kk * 2),
-                          b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, 1u);
-    }
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16_ss_elect(tmem + TM_S, a0 + static_cast<uint64_t>(kk * 2),
+                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, 1u);
+  }
+}
+// The score-only chunks of a tile (att_chunk_order j = 0..4): half 0 reads chunks 4,5 | 6,7,8,
+// half 1 chunks 0..3 | 8; the tile's first K-step overwrites S.
+__device__ __forceinline__ void att_qk_score_only(uint32_t tmem, uint64_t b_stage,
+                                                  uint64_t qs_desc, int half) {
+  if (half == 0) {
+    att_qk_ts(tmem, b_stage, 4, 2, true);
+    att_qk_ss(tmem, b_stage, qs_desc, 6, 3);
+  } else {
+    att_qk_ts(tmem, b_stage, 0, 4, true);
+    att_qk_ss(tmem, b_stage, qs_desc, 8, 1);
+  }
+}
+// This CTA's own chunks (j = 5..8): half 0 chunks 0..3, half 1 chunks 4,5 | 6,7.
+__device__ __forceinline__ void att_qk_own(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
+                                           int half) {
+  if (half == 0) {
+    att_qk_ts(tmem, b_stage, 0, 4, false);
+  } else {
+    att_qk_ts(tmem, b_stage, 4, 2, false);
+    att_qk_ss(tmem, b_stage, qs_desc, 6, 2);
   }
 }
 
@@ -490,11 +517,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           // S over the score-only chunks first, then this CTA's own chunks (see att_chunk_order)
           if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          att_qk_part(tmem, b_stage, qs_desc, half, 0, 5);
+          att_qk_score_only(tmem, b_stage, qs_desc, half);
           mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
           if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          att_qk_part(tmem, b_stage, qs_desc, half, 5, 9);
+          att_qk_own(tmem, b_stage, qs_desc, half);
           mma_commit_elect(&sh.s_full);
           if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
           mma_commit_elect(&sh.empty_own[st]);
