@@ -145,10 +145,59 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// Encoded maps are cached: a map is a pure function of (base, rank, dims, strides, box), so a
+// hit is always exact, and decode steps that reuse their buffers skip the driver call.
+struct MapKey {
+  uint64_t v[12];
+  bool operator==(const MapKey& o) const {
+    for (int i = 0; i < 12; ++i)
+      if (v[i] != o.v[i]) return false;
+    return true;
+  }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = 1469598103934665603ull;
+    for (int i = 0; i < 12; ++i) h = (h ^ k.v[i]) * 1099511628211ull;
+    return static_cast<size_t>(h);
+  }
+};
+constexpr size_t kMapCacheMax = 4096;
+
+bool encode_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box);
+
 // bf16 tensor map with 128-byte swizzle. dims[0] is the contiguous dimension; strides are the
 // byte strides of dims 1.. ; box[0] must be 64 (one 128-byte swizzle row).
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
               const uint64_t* strides_bytes, const uint32_t* box) {
+  static std::mutex mu;
+  static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  MapKey k{};
+  k.v[0] = reinterpret_cast<uint64_t>(base);
+  k.v[1] = static_cast<uint64_t>(rank);
+  for (int i = 0; i < rank && i < 3; ++i) {
+    k.v[2 + i] = dims[i];
+    k.v[5 + i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank && i < 2; ++i) k.v[8 + i] = strides_bytes[i];
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(k);
+    if (it != cache.end()) {
+      *m = it->second;
+      return true;
+    }
+  }
+  if (!encode_map(m, base, rank, dims, strides_bytes, box)) return false;
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= kMapCacheMax) cache.clear();
+  cache.emplace(k, *m);
+  return true;
+}
+
+bool encode_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
   cuuint64_t d[3], s[2];
