@@ -149,6 +149,36 @@ def test_decode_long_sequence_alone_and_in_batch():
     _decode_and_check(mixed, heads=[0, 64, 127])
 
 
+def test_decode_more_sequences_than_cta_pairs():
+    """160 short sequences: more units than CTA pairs, so pairs run several units each and
+    the planner's multi-segment ranges, empty-unit edges and pair starts are all exercised."""
+    g = torch.Generator().manual_seed(11)
+    lens = torch.randint(1, 300, (160,), generator=g, dtype=torch.int32)
+    lens[::37] = 1
+    c = Hs.make_case(W.small_variant(V2, B=160), lens)
+    _decode_and_check(c, heads=[0, 127], bs=list(range(0, 160, 9)) + [159])
+
+
+def test_decode_profiled_matches_decode_and_records_events():
+    """mla_decode_profiled computes exactly what mla_decode computes and records its four
+    events in order."""
+    w = W.small_variant(V2, B=3)
+    c = Hs.make_case(w, _lens(4097, 65, 300))
+    Hs.run_append(c)
+    ref = Hs.run_decode(c)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+    for e in ev:
+        e.record()
+    out = torch.empty_like(ref)
+    ws = mla.workspace(mla.mla_decode_workspace_size(c.cfg, w.B, w.Tq))
+    mla.mla_decode_profiled(c.cfg, c.d["q"], c.d["cache"], c.d["block_table"], c.d["seq_lens"],
+                            c.d["w_uk_t"], c.d["w_uv"], ws, out, ev)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    gaps = [ev[i].elapsed_time(ev[i + 1]) for i in range(3)]
+    assert all(t >= 0.0 for t in gaps) and gaps[1] > 0.0   # the attention kernel takes time
+
+
 @pytest.mark.parametrize("name", ["v2_bf16_b16_ctx4096", "h32_bf16_b32_ctx512to8192_shuffled",
                                   "v2_bf16_b64_ctx1kto32k_mix", "v2_bf16_b4_ctx131072_tq2"])
 def test_decode_full_size_sampled(name):
