@@ -202,6 +202,20 @@ def build_inputs(w: WL.Workload, device):
     return lens, pt, weights, cache_host, x_new, seq_idx, pos, q
 
 
+def max_over_ranks(x: float, world: int, device) -> float:
+    """The largest x over all ranks (the job's time is the slowest rank's); x itself at N=1."""
+    if world <= 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(units_per_rank: float, ms_per_step: float, world: int) -> float:
+    """Whole-job throughput: every rank processes its own units_per_rank each step."""
+    return world * units_per_rank / (ms_per_step / 1e3)
+
+
 def run_reference(args, rank: int, world: int):
     """Reference arm: the fp64 oracle on this host's cores, same workload / metric / unit."""
     if rank != 0:
@@ -356,13 +370,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for evs in prof_ev:
         for j, n in enumerate(names):
             per[n].append(evs[j].elapsed_time(evs[j + 1]))
-    total_ms = sum(steps_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(steps_ms), world, dev)
     ms_per_step = total_ms / K
-    value = world * work["units"] / (ms_per_step / 1e3)
+    value = job_rate(work["units"], ms_per_step, world)
     kernel_ms = {n: statistics.fmean(v) for n, v in per.items()}
     kernel_ms["marked_step"] = statistics.fmean(
         evs[0].elapsed_time(evs[4]) for evs in prof_ev)
@@ -401,11 +411,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         b.record()
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    e2e_step = statistics.fmean(e2e_ms)
-    if world > 1:
-        t = torch.tensor([e2e_step], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_step = float(t.item())
+    e2e_step = max_over_ranks(statistics.fmean(e2e_ms), world, dev)
     err = mla.mla_get_device_error()
     if err != 0:
         raise RuntimeError(f"device error in the e2e loop: {mla.mla_status_string(err)}")
@@ -456,7 +462,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "step": "mla_append_latent + mla_decode"},
         "roofline": roof,
         "kernel_ms": kernel_ms,
-        "e2e": {"value": world * work["units"] / (e2e_step / 1e3), "unit": UNIT,
+        "e2e": {"value": job_rate(work["units"], e2e_step, world), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step},
         "gpu_launches": K * 5,
         "clocks": clk,

@@ -1,0 +1,62 @@
+"""The N > 1 host logic of bench.py on CPU, with two gloo ranks: the job's step time is the
+slowest rank's, the job's rate sums every rank's units, and the reference arm runs on rank 0
+only (the other ranks return at once, without work or output)."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank: int, world: int, port: int, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        # rank r measured a step of 1 + r ms: the job took the slowest rank's time
+        t = bench.max_over_ranks(1.0 + rank, world, torch.device("cpu"))
+        rate = bench.job_rate(1000.0, t, world)
+        out[rank] = (t, rate)
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_take_the_slowest_rank_and_sum_the_work():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.spawn(_rank_main, args=(world, port, out), nprocs=world, join=True)
+        res = dict(out)
+    assert res[0] == res[1]
+    t, rate = res[0]
+    assert t == 2.0                          # slowest rank: 1 + (world - 1) ms
+    assert rate == pytest.approx(world * 1000.0 / 2e-3)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
+    assert bench.job_rate(10.0, 2.0, 1) == pytest.approx(5000.0)
+
+
+class _Args:   # the fields run_reference reads
+    workload = "v2_bf16_b16_ctx4096"
+    steps = 1
+    warmup = 0
+    gpus = 2
+
+
+def test_reference_arm_runs_on_rank_zero_only(capsys):
+    bench.run_reference(_Args(), rank=1, world=2)
+    assert capsys.readouterr().out == ""
