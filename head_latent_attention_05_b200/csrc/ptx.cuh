@@ -70,20 +70,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
-// Same wait with cluster-scope acquire: for phases completed by another CTA of the cluster
-// (remote arrives, st.async transactions).
-__device__ __forceinline__ bool mbar_try_wait_cluster(uint64_t* bar, uint32_t parity) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}\n"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity)
-      : "memory");
-  return done != 0;
-}
-
 // ------------------------------------------------------------------------ thread-block cluster
 
 __device__ __forceinline__ uint32_t cluster_ctarank() {
@@ -106,30 +92,6 @@ __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t cluster_addr) {
   return v;
 }
 
-// Asynchronous 16-byte store into another CTA's shared memory; on completion it performs a
-// complete_tx of 16 bytes on the mbarrier at `remote_bar` (in that same CTA).
-__device__ __forceinline__ void st_async_v4(uint32_t remote_addr, uint32_t a, uint32_t b,
-                                            uint32_t c, uint32_t d, uint32_t remote_bar) {
-  asm volatile(
-      "st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.b32 [%0], {%1, %2, %3, %4}, [%5];"
-      ::"r"(remote_addr), "r"(a), "r"(b), "r"(c), "r"(d), "r"(remote_bar)
-      : "memory");
-}
-
-// Arrive (release, cluster scope) on an mbarrier of another CTA of the cluster.
-__device__ __forceinline__ void mbar_arrive_remote(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
-}
-
-// Relaxed remote arrive: a pure "buffer consumed" signal that orders no memory accesses (the
-// data it guards has already been read into registers), so it does not wait for this thread's
-// earlier stores to complete.
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t remote_bar) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar)
-               : "memory");
-}
-
 // All threads of all CTAs of the cluster.
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile(
@@ -144,13 +106,6 @@ __device__ __forceinline__ uint64_t l2_policy_evict_last() {
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(pol));
   return pol;
 }
-__device__ __forceinline__ void st_global_v4_hint(float* dst, float a, float b, float c, float d,
-                                                  uint64_t pol) {
-  asm volatile("st.global.L2::cache_hint.v4.f32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "f"(a),
-               "f"(b), "f"(c), "f"(d), "l"(pol)
-               : "memory");
-}
-
 __device__ __forceinline__ void st_global_u4_hint(void* dst, uint32_t a, uint32_t b, uint32_t c,
                                                   uint32_t d, uint64_t pol) {
   asm volatile("st.global.L2::cache_hint.v4.b32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(dst), "r"(a),
@@ -219,40 +174,16 @@ __device__ __forceinline__ void tc_fence_after_sync() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (bf16 inputs, fp32 accumulate).
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// D[tmem] (+)= A[tmem] * B[smem desc]; A holds bf16 pairs packed in 32-bit columns.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
-// Arrive once on *bar when every tcgen05 operation issued so far by this thread completes.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-          smem_addr(bar))
-      : "memory");
-}
-
-// Warp-converged forms: every lane of a fully converged warp executes them and the one lane
-// that elect.sync picks (the same lane each time for the same converged warp) issues the MMA or
-// the commit. An issuing warp that stays converged like this issued N = 64 MMAs at ~37 cycles
-// each on B200 even with other warps busy; a single-lane, diverged issuer took 45-66.
+// tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), cta_group::1: D[tmem] = A * B (accumulate == 0)
+// or D += A * B. The _ss form takes A and B from shared memory (matrix descriptors), the _ts
+// form A from TMEM (bf16 pairs packed in 32-bit columns) and B from shared memory. The commit
+// arrives once on *bar when every tcgen05 operation issued so far by the issuing thread has
+// completed.
+// All three are warp-converged: every lane of a fully converged warp executes them and the one
+// lane that elect.sync picks (the same lane each time for the same converged warp) issues the
+// instruction, so MMAs and their commit come from one thread. An issuing warp that stays
+// converged like this issued N = 64 MMAs at ~37 cycles each on B200 even with other warps busy;
+// a single-lane, diverged issuer took 45-66.
 __device__ __forceinline__ void mma_bf16_ss_elect(uint32_t d_tmem, uint64_t a_desc,
                                                   uint64_t b_desc, uint32_t idesc,
                                                   uint32_t accumulate) {
@@ -308,16 +239,6 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
         "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
         "=r"(r[31])
       : "r"(taddr));
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-      "r"(r[15])
-      : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
@@ -376,13 +297,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn_major,
          | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
-// Byte offset of element (row, col) of a [rows x 64] bf16 tile stored K-major with the
-// 128-byte swizzle: 16-byte chunk index XOR (row % 8).
-__device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t col) {
-  const uint32_t chunk = (col >> 3) ^ (row & 7u);
-  return row * 128u + chunk * 16u + (col & 7u) * 2u;
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<uint32_t*>(&v);
@@ -394,8 +308,6 @@ __device__ __forceinline__ float fast_exp2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
-
-__device__ __forceinline__ bool elect_lane0() { return (threadIdx.x & 31u) == 0u; }
 
 // Programmatic dependent launch. A kernel launched with programmatic stream serialization may
 // start while the previous kernel of the stream still runs; pdl_wait() blocks until that kernel

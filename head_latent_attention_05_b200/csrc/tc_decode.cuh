@@ -295,11 +295,8 @@ struct TileCursor {
   }
 };
 
-// Chunk j of a tile in the order the score MMA consumes it: first the 5 chunks only it needs
-// (the other half's 4 c_KV chunks, then k_R), then this CTA's own 4 c_KV chunks.
-__device__ __forceinline__ int att_chunk_order(int half, int j) {
-  return j < 4 ? 4 * (1 - half) + j : (j == 4 ? 8 : 4 * half + (j - 5));
-}
+// The score MMA consumes a tile's chunks in two parts: first the 5 chunks only it needs (the
+// other half's 4 c_KV chunks, then k_R = chunk 8), then this CTA's own 4 c_KV chunks.
 
 // Score K-steps over a run of consecutive chunks c .. c+n-1 of a tile. In the A-from-TMEM form
 // (chunks below 6: Q̂[:, 0:384] sits in TMEM) and the A-from-smem form (Q̂[:, 384:576]). Each
@@ -333,7 +330,7 @@ __device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint64_t b_stage, uint6
                         b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, 1u);
   }
 }
-// The score-only chunks of a tile (att_chunk_order j = 0..4): half 0 reads chunks 4,5 | 6,7,8,
+// The score-only chunks of a tile: half 0 reads chunks 4,5 | 6,7,8,
 // half 1 chunks 0..3 | 8; the tile's first K-step overwrites S.
 __device__ __forceinline__ void att_qk_score_only(uint32_t tmem, uint64_t b_stage,
                                                   uint64_t qs_desc, int half) {
@@ -345,7 +342,7 @@ __device__ __forceinline__ void att_qk_score_only(uint32_t tmem, uint64_t b_stag
     att_qk_ss(tmem, b_stage, qs_desc, 8, 1);
   }
 }
-// This CTA's own chunks (j = 5..8): half 0 chunks 0..3, half 1 chunks 4,5 | 6,7.
+// This CTA's own chunks: half 0 chunks 0..3, half 1 chunks 4,5 | 6,7.
 __device__ __forceinline__ void att_qk_own(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
                                            int half) {
   if (half == 0) {
@@ -514,7 +511,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) break;
           if (g >= 1 && !att_warp_wait(sh, &sh.s_free, (g - 1) & 1)) break;
           const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
-          // S over the score-only chunks first, then this CTA's own chunks (see att_chunk_order)
+          // S over the score-only chunks first, then this CTA's own chunks
           if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
           att_qk_score_only(tmem, b_stage, qs_desc, half);
