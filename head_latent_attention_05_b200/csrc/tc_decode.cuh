@@ -84,7 +84,7 @@ struct AttnParams {
   float scale_log2;          // softmax_scale * log2(e)
 };
 
-// ------------------------------------------------------------------------ planning kernel
+// ------------------------------------------------------------------------ split-KV planner
 
 struct PlanParams {
   const int32_t* seq_lens;
