@@ -61,7 +61,6 @@ constexpr int ATT_SMEM_BYTES =
     ATT_STAGES * ATT_TILE_BYTES + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES + ATT_P_BYTES + 1024;
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;     // log2 units
-constexpr int ATT_PREFETCH_AHEAD = 4;             // pages prefetched into L2 ahead of the loads
 
 struct AttnSeg {
   int32_t unit;        // b * n_mt + mt
@@ -76,7 +75,6 @@ struct AttnParams {
   const AttnSeg* segs;
   const int32_t* pair_seg;   // [P + 1]: pair p runs segments [pair_seg[p], pair_seg[p+1])
   const __nv_bfloat16* qhat; // [B*R][576]
-  const __nv_bfloat16* cache;  // [num_pages][64][576] (for L2 prefetch)
   __nv_bfloat16* o_part;     // [max_segs][128][512] per-segment O / l, rounded to bf16
   float* lse;                // [max_segs][128]   (base-2 log-sum-exp of the scaled scores)
   int max_pages, num_pages;
@@ -438,17 +436,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         // Step for tile g: its own chunks, then (new segment at g+1) the next Q̂, then the
         // score-only chunks of tile g+1. Own chunks of g wait for P·C of g-2; score-only chunks
         // of g+1 wait for S of g-1, which completes earlier, so neither load delays the other.
-        TileCursor cq, co, cp;   // score-only cursor (one tile ahead), own-chunk cursor,
-        cq.init(p.segs, seg_begin, seg_end);   // L2-prefetch cursor (further ahead, half 0 only)
+        // (No L2 prefetch of pages ahead of these loads: the TMA engine that would issue it is
+        // the one these loads wait on, and on B200 it measured no faster with it.)
+        TileCursor cq, co;   // score-only cursor (one tile ahead), own-chunk cursor
+        cq.init(p.segs, seg_begin, seg_end);
         co.init(p.segs, seg_begin, seg_end);
-        cp.init(p.segs, seg_begin, seg_end);
-        auto prefetch_next = [&]() {
-          if (half != 0 || !cp.valid()) return;
-          prefetch_l2_bulk(p.cache + static_cast<int64_t>(page_of(cp)) * ATT_PAGE * ATT_ROW,
-                           ATT_TILE_BYTES);
-          cp.next();
-        };
-        for (int i = 0; i < ATT_PREFETCH_AHEAD; ++i) prefetch_next();
         // Q̂ rows of this pair's later segments into L2 now, so that switching units later
         // reads them from L2 rather than HBM
         if (half == 0) {
@@ -490,7 +482,6 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           load_chunks(cq, gq, false, &sh.full_qk[st]);
           cq.next();
           ++gq;
-          prefetch_next();
         }
         // drain: the last loads must land before the CTA can exit (bounded, abort or not)
         for (int j = max(0, gq - ATT_STAGES); j < gq; ++j)
