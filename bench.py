@@ -284,8 +284,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     step_ev = [[ev() for _ in range(2)] for _ in range(K)]
     # breakdown replay: start, the 4 decode marks (absorption, attention, merge+projection, end)
     prof_ev = [[ev() for _ in range(5)] for _ in range(K)]
+    # decode-only replay: events around mla_decode alone (the roofline's definition of the path)
+    dec_ev = [[ev() for _ in range(2)] for _ in range(K)]
     # torch creates events lazily: record every event once so it exists before capture
-    for evs in step_ev + prof_ev:
+    for evs in step_ev + prof_ev + dec_ev:
         for e in evs:
             e.record()
     torch.cuda.synchronize()
@@ -333,10 +335,18 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             flush_l2(i * 7)
             step(marks=prof_ev[i])
 
-    graph = graph_prof = None
+    def decode_steps():
+        for i in range(K):
+            flush_l2(i * 7)
+            dec_ev[i][0].record()
+            mla.mla_decode(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out)
+            dec_ev[i][1].record()
+
+    graph = graph_prof = graph_dec = None
     if not args.no_graph:
         graph = capture(timed_steps)
         graph_prof = capture(marked_steps)
+        graph_dec = capture(decode_steps)
 
     clocks = ClockSampler(local_rank)
     clocks.start()
@@ -357,11 +367,13 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     err = mla.mla_get_device_error()
     if err != 0:
         raise RuntimeError(f"device error in the timed region: {mla.mla_status_string(err)}")
-    # the breakdown replay (same steps, event marks between the kernels)
+    # the breakdown replay (same steps, event marks between the kernels), then decode alone
     if graph_prof is not None:
         graph_prof.replay()
+        graph_dec.replay()
     else:
         marked_steps()
+        decode_steps()
     torch.cuda.synchronize()
 
     names = ["append", "q_absorb_plan", "attention", "merge_value_proj"]
@@ -376,6 +388,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     kernel_ms = {n: statistics.fmean(v) for n, v in per.items()}
     kernel_ms["marked_step"] = statistics.fmean(
         evs[0].elapsed_time(evs[4]) for evs in prof_ev)
+    decode_ms = max_over_ranks(statistics.fmean(e[0].elapsed_time(e[1]) for e in dec_ev), world,
+                               dev)
 
     # ---- e2e through the plain API from pinned host memory: the step's inputs are staged in
     # one pinned buffer and sent with one copy (as a serving loop would), the output comes back
@@ -447,6 +461,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         (work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
         (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12)) / (ms_per_step / 1e3)
 
+    # mla_decode alone against the path's roofline: the larger of (cache + W_UK + W_UV bytes)
+    # over HBM bandwidth and (attention + projection FLOPs) over the tensor peak
+    t_roof = max((work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
+                 (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12))
+    decode_only = {"value": job_rate(work["units"], decode_ms, world), "unit": UNIT,
+                   "ms_per_step": decode_ms, "roofline_frac": t_roof / (decode_ms / 1e3),
+                   "roofline_ms": t_roof * 1e3,
+                   "what": "mla_decode alone (query absorption + planner, attention, merge + "
+                           "value projection), same L2 flush, graph-timed"}
+
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": Wm, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
@@ -462,6 +486,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                    "step": "mla_append_latent + mla_decode"},
         "roofline": roof,
         "kernel_ms": kernel_ms,
+        "decode_only": decode_only,
         "e2e": {"value": job_rate(work["units"], e2e_step, world), "unit": UNIT,
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step},
         "gpu_launches": K * 5,
@@ -476,7 +501,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                 "kind": "oracle", "sample": desc}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_prof
+    del graph, graph_prof, graph_dec
 
 
 def kernel_sha() -> str:
