@@ -159,10 +159,12 @@ def cpu_threads() -> int:
 # ------------------------------------------------------------------ oracle (CPU baseline)
 
 def oracle_sample(w: WL.Workload, lens, pt, weights, cache_host, x_new, pos, q, seconds: float,
-                  max_units: int | None = None):
-    """Time the fp64 oracle (expanded form, as it stands) on (sequence, head) units of the
-    workload for about `seconds`; returns (rate in cache-tokens*heads/s, units, description)."""
+                  max_units: int | None = None, form: str = "expanded"):
+    """Time the fp64 oracle (as it stands; the expanded form unless form == "absorbed") on
+    (sequence, head) units of the workload for about `seconds`; returns (rate in
+    cache-tokens*heads/s, units, description)."""
     from oracle import mla_oracle as O
+    decode = O.decode_absorbed if form == "absorbed" else O.decode_expanded
     W_UK, W_UV = O.split_wkv_b(weights.wkv_b, w.H, w.d_nope, w.d_v)
     new_rows = O.latent_rows(x_new, weights.w_dkv, weights.kv_gain, pos.numpy(), w.d_c,
                              w.rms_eps, w.rope_theta)
@@ -180,12 +182,12 @@ def oracle_sample(w: WL.Workload, lens, pt, weights, cache_host, x_new, pos, q, 
             r[L - w.Tq:] = new_rows[b * w.Tq:(b + 1) * w.Tq]
             rows_cache = {b: r}
         t0 = time.perf_counter()
-        O.decode_expanded(q[b], rows_cache[b], W_UK, W_UV, w.scale, w.rope_theta, heads=[h])
+        decode(q[b], rows_cache[b], W_UK, W_UV, w.scale, w.rope_theta, heads=[h])
         elapsed += time.perf_counter() - t0
         done_units += 1
         done_work += L * w.Tq
     rate = done_work / elapsed if elapsed > 0 else 0.0
-    desc = (f"{done_units} (sequence, head) units of {w.name} through the fp64 expanded-form "
+    desc = (f"{done_units} (sequence, head) units of {w.name} through the fp64 {form}-form "
             f"oracle ({done_work} cache-token*heads, {elapsed:.1f} s); rate scales to the full "
             f"workload because the work per cache-token*head is uniform")
     return rate, done_units, desc
@@ -499,6 +501,11 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                           args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cpu_threads(),
                                 "kind": "oracle", "sample": desc}
+        # the same oracle's absorbed (latent-space) form, a second CPU number
+        rate_a, _, desc_a = oracle_sample(w, lens, pt, weights, cache_host, x_new_h, pos_h, q_h,
+                                          args.cpu_seconds / 3, form="absorbed")
+        line["cpu_baseline_absorbed"] = {"value": rate_a, "unit": UNIT, "cores": cpu_threads(),
+                                         "kind": "oracle", "sample": desc_a}
     if rank == 0:
         print(json.dumps(line), flush=True)
     del graph, graph_prof, graph_dec

@@ -1,6 +1,7 @@
-"""The N > 1 host logic of bench.py on CPU, with two gloo ranks: the job's step time is the
-slowest rank's, the job's rate sums every rank's units, and the reference arm runs on rank 0
-only (the other ranks return at once, without work or output)."""
+"""The host logic of bench.py on CPU. With two gloo ranks: the job's step time is the slowest
+rank's, the job's rate sums every rank's units, and the reference arm runs on rank 0 only (the
+other ranks return at once, without work or output). And the CPU baseline's oracle sampler in
+both of the oracle's forms."""
 
 import os
 import socket
@@ -60,3 +61,12 @@ class _Args:   # the fields run_reference reads
 def test_reference_arm_runs_on_rank_zero_only(capsys):
     bench.run_reference(_Args(), rank=1, world=2)
     assert capsys.readouterr().out == ""
+
+
+@pytest.mark.parametrize("form", ["expanded", "absorbed"])
+def test_oracle_sample_times_both_forms(form):
+    w = bench.WL.WORKLOADS["tiny_f32_b1_h4_ctx128"]
+    lens, pt, weights, cache_host, x_new, seq_idx, pos, q = bench.build_inputs(w, "cpu")
+    rate, units, desc = bench.oracle_sample(w, lens, pt, weights, cache_host, x_new, pos, q,
+                                            float("inf"), max_units=3, form=form)
+    assert units == 3 and rate > 0.0 and form in desc
