@@ -62,6 +62,7 @@ def test_decode_rejects_bad_arguments(lib):
     assert _decode(lib, cfg, tq=0) == 1
     assert _decode(lib, _cfg(n_heads=0)) == 1                   # bad config
     assert _decode(lib, _cfg(d_rope=63)) == 1                   # odd rope width
+    assert _decode(lib, _cfg(d_rope=130, d_c=510)) == 2         # rope wider than 128
     assert _decode(lib, _cfg(d_c=256)) == 2                     # bf16 path is V2-shaped only
     assert _decode(lib, cfg, ws_bytes=16) == 3                  # workspace too small
     assert lib.mla_decode(None, FAKE, 1, 1, FAKE, 1, FAKE, 1, FAKE, FAKE, FAKE, FAKE, 1, FAKE,
