@@ -70,3 +70,21 @@ def test_oracle_sample_times_both_forms(form):
     rate, units, desc = bench.oracle_sample(w, lens, pt, weights, cache_host, x_new, pos, q,
                                             float("inf"), max_units=3, form=form)
     assert units == 3 and rate > 0.0 and form in desc
+
+
+def test_reference_arm_prints_one_json_line():
+    """`bench.py --impl reference` (the fp64 oracle on the host) runs without a GPU and prints
+    the contract's line: metric, value, unit, impl, cpu_baseline and a zero-copy e2e."""
+    import json
+    import subprocess
+    import sys
+    r = subprocess.run([sys.executable, "bench.py", "--impl", "reference", "--workload",
+                        "tiny_f32_b1_h4_ctx128", "--steps", "2", "--warmup", "1"],
+                       cwd=bench.ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == bench.UNIT
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
