@@ -27,6 +27,12 @@
  *     outputs are zero-filled, no memory outside the given buffers is touched, and the next
  *     mla_get_device_error call reports the first such error.
  *   - Calls that share a workspace or a cache must not overlap on the GPU (use one stream).
+ *   - Within a call, kernels after the first are launched with programmatic dependent launch
+ *     and let the next kernel of the stream start early. A caller's own kernel enqueued right
+ *     after a call with programmatic stream serialization must therefore wait
+ *     (griddepcontrol.wait / cudaGridDependencySynchronize) before reading the call's
+ *     outputs; kernels launched the ordinary way are unaffected. The first kernel of every
+ *     call is launched the ordinary way, so the call sees all earlier work on the stream.
  */
 #ifndef MLA_H_
 #define MLA_H_
