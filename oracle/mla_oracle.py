@@ -16,7 +16,8 @@ Readings where the pages are silent (each is also listed in the design notes):
   * positions are 0-based; query t of Tq new tokens sits at position L - Tq + t;
   * the new tokens are appended before attending, so a query sees itself;
   * RMSNorm is x / sqrt(mean(x^2) + eps) * gain, applied to c_KV only (not to k_R);
-  * the output stops before the output projection wo.
+  * decode_expanded stops before the output projection wo; output_projection applies it and
+    decode_layer chains the whole layer (q path, append, attention, wo).
 All arithmetic is float64; bf16 inputs are promoted exactly.
 """
 
@@ -191,6 +192,41 @@ def module_attention(x, w_dkv, kv_gain, wkv_b, w_qa, q_gain, w_qb, H, d_c, d_r, 
     rows = latent_rows(x, w_dkv, kv_gain, np.arange(L), d_c, eps, theta)
     W_UK, W_UV = split_wkv_b(wkv_b, H, d_nope, d_v)
     return decode_expanded(q, rows, W_UK, W_UV, 1.0 / np.sqrt(d_nope + d_r), theta)
+
+
+def output_projection(out, w_o) -> np.ndarray:
+    """The module's output projection wo applied to per-head attention outputs.
+
+    「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2: the heads' outputs are laid side by side,
+    head after head (transpose to (seq, heads, d_v), then view as heads * d_v), and wo, an
+    nn.Linear(heads * d_v, dim) without bias, maps them back to the model width.
+    out [..., H, d_v], w_o [d_model, H * d_v]; returns [..., d_model].
+    """
+    out = f64(out)
+    flat = out.reshape(out.shape[:-2] + (out.shape[-2] * out.shape[-1],))
+    return flat @ f64(w_o).T
+
+
+def decode_layer(x_new, rows_hist, w_dkv, kv_gain, wkv_b, w_qa, q_gain, w_qb, w_o, H: int,
+                 d_c: int, d_r: int, d_nope: int, d_v: int, eps: float, theta: float):
+    """One decode step of the whole attention layer for one sequence, expanded form.
+
+    x_new [Tq, d_model] are the hidden states of the Tq new tokens; rows_hist [L - Tq, d_c+d_r]
+    the cache rows already stored for the sequence. Steps, in the order of the page's module
+    (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2): the q path wq_a -> q_norm -> wq_b; the
+    new tokens' latent rows appended at positions L - Tq .. L - 1; attention of the new tokens
+    over all L rows (each sees itself and earlier tokens); the output projection wo.
+    Returns y [Tq, d_model].
+    """
+    x_new = f64(x_new)
+    Tq = x_new.shape[0]
+    L = rows_hist.shape[0] + Tq
+    q = query_from_x(x_new, w_qa, q_gain, w_qb, H, d_nope, d_r, eps)
+    new_rows = latent_rows(x_new, w_dkv, kv_gain, np.arange(L - Tq, L), d_c, eps, theta)
+    rows = np.concatenate([f64(rows_hist), new_rows], axis=0)
+    W_UK, W_UV = split_wkv_b(wkv_b, H, d_nope, d_v)
+    out = decode_expanded(q, rows, W_UK, W_UV, 1.0 / np.sqrt(d_nope + d_r), theta)
+    return output_projection(out, w_o)
 
 
 def gather_rows(cache, block_table_row, L: int, page_size: int = 64) -> np.ndarray:

@@ -329,3 +329,85 @@ def test_cache_sizes_page4_gqa():
     assert round(e / O.mla_cache_elems_per_token(512, 64)) == q["times_mla_approx"]
     gib = e * v2["layers"] * v2["bytes_per_elem"] * v2["context"] / 2 ** 30
     assert _close(gib, q["GiB_32k_approx"], q["rel_tol"])
+
+
+# --------------------------------------------------------------- output projection and layer
+
+def _brute_wo(out, w_o):
+    """Scalar loops: y[t][m] = sum over heads h and value dims k of w_o[m][h*d_v + k] out[t][h][k]."""
+    L, H, d_v = len(out), len(out[0]), len(out[0][0])
+    return np.array([[sum(w_o[m][h * d_v + k] * out[t][h][k] for h in range(H) for k in range(d_v))
+                      for m in range(len(w_o))] for t in range(L)])
+
+
+def test_output_projection_brute_force():
+    rng = np.random.default_rng(20)
+    dims = dict(H=3, d_c=6, d_r=4, d_nope=3, d_v=2)
+    d_model, q_lora, L, eps, theta = 5, 4, 6, 1e-6, 10000.0
+    W = _rand_module(rng, d_model, q_lora=q_lora, **dims)
+    w_o = rng.standard_normal((d_model, dims["H"] * dims["d_v"]))
+    x = rng.standard_normal((L, d_model))
+    attn = _brute_module(x.tolist(), W, eps=eps, theta=theta, **dims)
+    ref = _brute_wo(attn.tolist(), w_o.tolist())
+    got = O.output_projection(O.module_attention(x, W["w_dkv"], W["kv_gain"], W["wkv_b"],
+                                                 W["w_qa"], W["q_gain"], W["w_qb"], eps=eps,
+                                                 theta=theta, **dims), w_o)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_output_projection_flattens_head_after_head():
+    """Identity wo returns the heads laid side by side; a one-hot row picks (head 1, dim 0)."""
+    rng = np.random.default_rng(21)
+    out = rng.standard_normal((2, 3, 4))                      # [Tq, H, d_v]
+    np.testing.assert_array_equal(O.output_projection(out, np.eye(12)), out.reshape(2, 12))
+    w_o = np.zeros((1, 12))
+    w_o[0, 1 * 4 + 0] = 1.0
+    np.testing.assert_array_equal(O.output_projection(out, w_o)[:, 0], out[:, 1, 0])
+
+
+def test_output_projection_matches_torch_linear_on_the_module():
+    rng = np.random.default_rng(22)
+    dims = dict(H=4, d_c=32, d_r=8, d_nope=16, d_v=12)
+    d_model, q_lora, L = 24, 16, 30
+    W = _rand_module(rng, d_model, q_lora=q_lora, **dims)
+    w_o = rng.standard_normal((d_model, dims["H"] * dims["d_v"])) / math.sqrt(48)
+    x = rng.standard_normal((L, d_model))
+    o = torch.as_tensor(_torch_module(x, W, eps=1e-6, theta=10000.0, **dims))
+    ref = F.linear(o.reshape(L, -1), torch.as_tensor(w_o)).numpy()
+    got = O.output_projection(O.module_attention(x, W["w_dkv"], W["kv_gain"], W["wkv_b"],
+                                                 W["w_qa"], W["q_gain"], W["w_qb"], eps=1e-6,
+                                                 theta=10000.0, **dims), w_o)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("Tq", [1, 3])
+def test_decode_layer_equals_brute_force_prefill_tail(Tq):
+    """The whole decode layer for the Tq newest tokens (q path, append at their positions,
+    attention, wo) equals the last Tq rows of the brute-force module over the whole sequence."""
+    rng = np.random.default_rng(23 + Tq)
+    dims = dict(H=2, d_c=6, d_r=4, d_nope=3, d_v=2)
+    d_model, q_lora, L, eps, theta = 5, 4, 7, 1e-6, 300.0
+    W = _rand_module(rng, d_model, q_lora=q_lora, **dims)
+    w_o = rng.standard_normal((d_model, dims["H"] * dims["d_v"]))
+    x = rng.standard_normal((L, d_model))
+    ref = _brute_wo(_brute_module(x.tolist(), W, eps=eps, theta=theta, **dims).tolist(),
+                    w_o.tolist())[-Tq:]
+    hist = O.latent_rows(x[:L - Tq], W["w_dkv"], W["kv_gain"], np.arange(L - Tq), dims["d_c"],
+                         eps, theta)
+    got = O.decode_layer(x[L - Tq:], hist, W["w_dkv"], W["kv_gain"], W["wkv_b"], W["w_qa"],
+                         W["q_gain"], W["w_qb"], w_o, eps=eps, theta=theta, **dims)
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-13)
+
+
+def test_query_path_brute_force():
+    """q = wq_b(q_norm(wq_a(x))) per head, by scalar loops, against query_from_x."""
+    rng = np.random.default_rng(25)
+    H, d_nope, d_r, d_model, q_lora, eps = 2, 3, 4, 6, 5, 1e-6
+    W = _rand_module(rng, d_model, H=H, d_c=4, d_r=d_r, d_nope=d_nope, d_v=2, q_lora=q_lora)
+    x = rng.standard_normal(d_model)
+    qa = [sum(W["w_qa"][o, i] * x[i] for i in range(d_model)) for o in range(q_lora)]
+    ms = sum(v * v for v in qa) / q_lora
+    qn = [qa[i] / math.sqrt(ms + eps) * W["q_gain"][i] for i in range(q_lora)]
+    q = [sum(W["w_qb"][o, i] * qn[i] for i in range(q_lora)) for o in range(H * (d_nope + d_r))]
+    got = O.query_from_x(x, W["w_qa"], W["q_gain"], W["w_qb"], H, d_nope, d_r, eps)
+    np.testing.assert_allclose(got, np.array(q).reshape(H, d_nope + d_r), rtol=1e-12, atol=1e-13)

@@ -170,6 +170,13 @@ def weights(w: Workload) -> Weights:
     )
 
 
+def output_weight(w: Workload) -> torch.Tensor:
+    """wo weight [d_model, H*d_v] ~ N(0, 1/(H*d_v)), in dtype (drawn only when asked for: it is
+    the largest tensor of the layer, 168 MB in bf16 at DeepSeek-V2 shape)."""
+    return randn((w.d_model, w.H * w.d_v), w.seed, 14, 1.0 / math.sqrt(w.H * w.d_v),
+                 w.torch_dtype)
+
+
 def cache_pool(w: Workload, num_pages: int, chunk_pages: int = 2048) -> torch.Tensor:
     """Page pool [num_pages, 64, d_c+d_r] filled i.i.d. N(0,1) (the history rows), in dtype."""
     out = torch.empty((num_pages, PAGE_SIZE, w.row), dtype=w.torch_dtype)
