@@ -44,7 +44,9 @@ import workloads as WL  # noqa: E402
 
 METRIC = "MLA decode cache-tokens/s (×heads) on 1 B200; % of HBM/tensor roofline"
 UNIT = "cache_tokens*heads/s"
-DEFAULT_WORKLOAD = "v2_bf16_b16_ctx4096"
+DEFAULT_WORKLOAD = "v2_bf16_b64_ctx1kto32k_mix"
+# measured after the headline, each with its own attention roofline
+EXTRA_WORKLOADS = ("v2_bf16_b16_ctx4096", "v2_bf16_b4_ctx131072_tq2")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_PROFILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
 
@@ -60,6 +62,10 @@ def parse_args():
                     help="budget of the oracle CPU-baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the other workloads measured after the headline")
+    ap.add_argument("--extra-steps", type=int, default=40,
+                    help="timed steps of each extra workload")
     return ap.parse_args()
 
 
@@ -246,79 +252,131 @@ def run_reference(args, rank: int, world: int):
     print(json.dumps(line), flush=True)
 
 
-def run_ours(args, rank: int, world: int, local_rank: int):
-    import head_latent_attention_05_b200 as mla
+class DeviceCase:
+    """One workload's inputs on the device, the library's buffers and the step functions."""
 
-    dev = torch.device("cuda", local_rank)
-    torch.cuda.set_device(dev)
-    w = WL.WORKLOADS[args.workload]
-    lens, pt, weights, cache_host, x_new_h, seq_idx_h, pos_h, q_h = build_inputs(w, dev)
-    cfg = mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, WL.PAGE_SIZE, w.dtype,
-                          w.scale, w.rms_eps, w.rope_theta)
-    dt = w.torch_dtype
-    cache = cache_host.to(dev)
-    bt = pt.block_table.to(dev)
-    seq_lens = lens.to(dev)
-    x_new, seq_idx, pos, q = (t.contiguous().to(dev) for t in (x_new_h, seq_idx_h, pos_h, q_h))
-    w_dkv, kv_gain = weights.w_dkv.to(dev), weights.kv_gain.to(dev)
-    w_uk_t = torch.empty((w.H, w.d_c, w.d_nope), dtype=dt, device=dev)
-    w_uv = torch.empty((w.H, w.d_v, w.d_c), dtype=dt, device=dev)
-    mla.mla_absorb_weights(cfg, weights.wkv_b.to(dev), w_uk_t, w_uv)
-    n_tok = w.B * w.Tq
-    ws_a = mla.workspace(mla.mla_append_workspace_size(cfg, n_tok), dev)
-    ws_d = mla.workspace(mla.mla_decode_workspace_size(cfg, w.B, w.Tq), dev)
-    out = torch.empty((w.B, w.Tq, w.H, w.d_v), dtype=dt, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
-    drain = torch.zeros_like(flush)
+    def __init__(self, mla, w: WL.Workload, dev):
+        self.w, self.dev = w, dev
+        (self.lens, self.pt, self.weights, self.cache_host, self.x_new_h, self.seq_idx_h,
+         self.pos_h, self.q_h) = build_inputs(w, dev)
+        self.cfg = mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, WL.PAGE_SIZE,
+                                   w.dtype, w.scale, w.rms_eps, w.rope_theta)
+        dt = w.torch_dtype
+        self.cache = self.cache_host.to(dev)
+        self.bt = self.pt.block_table.to(dev)
+        self.seq_lens = self.lens.to(dev)
+        self.x_new, self.seq_idx, self.pos, self.q = (
+            t.contiguous().to(dev) for t in (self.x_new_h, self.seq_idx_h, self.pos_h, self.q_h))
+        self.w_dkv, self.kv_gain = self.weights.w_dkv.to(dev), self.weights.kv_gain.to(dev)
+        self.w_uk_t = torch.empty((w.H, w.d_c, w.d_nope), dtype=dt, device=dev)
+        self.w_uv = torch.empty((w.H, w.d_v, w.d_c), dtype=dt, device=dev)
+        mla.mla_absorb_weights(self.cfg, self.weights.wkv_b.to(dev), self.w_uk_t, self.w_uv)
+        n_tok = w.B * w.Tq
+        self.ws_a = mla.workspace(mla.mla_append_workspace_size(self.cfg, n_tok), dev)
+        self.ws_d = mla.workspace(mla.mla_decode_workspace_size(self.cfg, w.B, w.Tq), dev)
+        self.out = torch.empty((w.B, w.Tq, w.H, w.d_v), dtype=dt, device=dev)
+        self.work = work_of(w, self.lens)
+        self.mla = mla
 
-    def flush_l2(i):
-        # write a buffer twice the L2 size (the step's inputs leave L2), then read another one
-        # as large, so that the written buffer's dirty lines are drained to HBM here and not
-        # inside the next step
-        flush.fill_(i & 0xFF)
-        drain.max()
-    work = work_of(w, lens)
+    def step(self, evs=None, marks=None):
+        mla = self.mla
+        if evs is not None:
+            evs[0].record()
+        if marks is not None:
+            marks[0].record()
+        mla.mla_append_latent(self.cfg, self.x_new, self.w_dkv, self.kv_gain, self.seq_idx,
+                              self.pos, self.bt, self.cache, self.ws_a)
+        if marks is not None:
+            mla.mla_decode_profiled(self.cfg, self.q, self.cache, self.bt, self.seq_lens,
+                                    self.w_uk_t, self.w_uv, self.ws_d, self.out, marks[1:5])
+        else:
+            self.decode()
+        if evs is not None:
+            evs[1].record()
 
-    K, Wm = args.steps, max(3, args.warmup)
+    def decode(self):
+        self.mla.mla_decode(self.cfg, self.q, self.cache, self.bt, self.seq_lens, self.w_uk_t,
+                            self.w_uv, self.ws_d, self.out)
+
+
+class L2Flush:
+    """Before a step: write a buffer twice the L2 size (the step's inputs leave L2), then read
+    another as large, so that the written buffer's dirty lines drain to HBM here and not inside
+    the next step."""
+
+    def __init__(self, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        self.flush = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+        self.drain = torch.zeros_like(self.flush)
+
+    def __call__(self, i):
+        self.flush.fill_(i & 0xFF)
+        self.drain.max()
+
+
+def attn_roofline(w: WL.Workload, work: dict, t_attn_s: float, ms_per_step: float) -> dict:
+    """Roofline block of the latent attention kernel: its algorithmic bytes (or FLOPs) over its
+    own CUDA-event time, against the measured HBM copy rate (or bf16 tensor peak)."""
+    pk, pk_kind = peaks()
+    hbm_peak = float(pk["hbm_gbs"])
+    tc_peak = float(pk["bf16_tflops"])
+    t_mem = work["cache_bytes"] / (hbm_peak * 1e9)
+    t_tc = work["attn_flops"] / (tc_peak * 1e12)
+    bound = "hbm" if t_mem >= t_tc else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": work["cache_bytes"] / t_attn_s / 1e9,
+                "peak": hbm_peak, "unit": "GB/s"}
+    else:
+        roof = {"bound": "tensor", "achieved": work["attn_flops"] / t_attn_s / 1e12,
+                "peak": tc_peak, "unit": "TFLOP/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = stored_traffic(w.name)
+    roof["peak_source"] = (f"{pk_kind} (MEASURED_PEAKS.json: burst bf16 GEMM, copy HBM)"
+                           if pk_kind == "measured" else "fallback")
+    roof["kernel"] = "mla_decode_attn_kernel"
+    roof["kernel_us"] = t_attn_s * 1e6
+    roof["algorithmic_bytes_per_launch"] = work["cache_bytes"]
+    roof["algorithmic_flops_per_launch"] = work["attn_flops"]
+    roof["hbm_frac"] = (work["cache_bytes"] / t_attn_s / 1e9) / hbm_peak
+    roof["tensor_frac"] = (work["attn_flops"] / t_attn_s / 1e12) / tc_peak
+    roof["step_roofline_frac"] = max(
+        (work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
+        (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12)) / (ms_per_step / 1e3)
+    return roof
+
+
+def decode_roofline_ms(work: dict) -> float:
+    """The path's roofline time for mla_decode: the larger of (cache + W_UK + W_UV bytes) over
+    the HBM rate and (attention + projection FLOPs) over the tensor peak."""
+    pk, _ = peaks()
+    return 1e3 * max((work["cache_bytes"] + work["weight_bytes"]) / (float(pk["hbm_gbs"]) * 1e9),
+                     (work["attn_flops"] + work["proj_flops"]) / (float(pk["bf16_tflops"]) * 1e12))
+
+
+def measure_device(c: DeviceCase, flush_l2: L2Flush, K: int, Wm: int, world: int, use_graph: bool,
+                   local_rank: int):
+    """Warm up, then time K steps (append + decode) with CUDA events around each step, a marked
+    replay for the per-kernel breakdown and a decode-only replay. Returns a dict of results."""
+    mla = c.mla
     ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
-    # headline: one start and one end event per step, nothing between the kernels
     step_ev = [[ev() for _ in range(2)] for _ in range(K)]
-    # breakdown replay: start, the 4 decode marks (absorption, attention, merge+projection, end)
     prof_ev = [[ev() for _ in range(5)] for _ in range(K)]
-    # decode-only replay: events around mla_decode alone (the roofline's definition of the path)
     dec_ev = [[ev() for _ in range(2)] for _ in range(K)]
     # torch creates events lazily: record every event once so it exists before capture
     for evs in step_ev + prof_ev + dec_ev:
         for e in evs:
             e.record()
     torch.cuda.synchronize()
-
-    def step(evs=None, marks=None):
-        if evs is not None:
-            evs[0].record()
-        if marks is not None:
-            marks[0].record()
-        mla.mla_append_latent(cfg, x_new, w_dkv, kv_gain, seq_idx, pos, bt, cache, ws_a)
-        if marks is not None:
-            mla.mla_decode_profiled(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out,
-                                    marks[1:5])
-        else:
-            mla.mla_decode(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out)
-        if evs is not None:
-            evs[1].record()
-
-    # warm-up (eager), then a correctness guard: no device error may be pending
     for i in range(Wm):
         flush_l2(i)
-        step()
+        c.step()
     err = mla.mla_get_device_error()
     if err != 0:
         raise RuntimeError(f"device error during warm-up: {mla.mla_status_string(err)}")
 
     def capture(fn):
         g = torch.cuda.CUDAGraph()
-        s = torch.cuda.Stream(device=dev)
+        s = torch.cuda.Stream(device=c.dev)
         s.wait_stream(torch.cuda.current_stream())
         with torch.cuda.stream(s):
             with torch.cuda.graph(g, stream=s):
@@ -330,26 +388,21 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def timed_steps():
         for i in range(K):
             flush_l2(i * 7)
-            step(evs=step_ev[i])
+            c.step(evs=step_ev[i])
 
     def marked_steps():
         for i in range(K):
             flush_l2(i * 7)
-            step(marks=prof_ev[i])
+            c.step(marks=prof_ev[i])
 
     def decode_steps():
         for i in range(K):
             flush_l2(i * 7)
             dec_ev[i][0].record()
-            mla.mla_decode(cfg, q, cache, bt, seq_lens, w_uk_t, w_uv, ws_d, out)
+            c.decode()
             dec_ev[i][1].record()
 
-    graph = graph_prof = graph_dec = None
-    if not args.no_graph:
-        graph = capture(timed_steps)
-        graph_prof = capture(marked_steps)
-        graph_dec = capture(decode_steps)
-
+    graphs = [capture(f) for f in (timed_steps, marked_steps, decode_steps)] if use_graph else None
     clocks = ClockSampler(local_rank)
     clocks.start()
     time.sleep(0.03)
@@ -357,8 +410,8 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     t_wall0 = time.perf_counter()
-    if graph is not None:
-        graph.replay()
+    if graphs is not None:
+        graphs[0].replay()
     else:
         timed_steps()
     torch.cuda.synchronize()
@@ -370,13 +423,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if err != 0:
         raise RuntimeError(f"device error in the timed region: {mla.mla_status_string(err)}")
     # the breakdown replay (same steps, event marks between the kernels), then decode alone
-    if graph_prof is not None:
-        graph_prof.replay()
-        graph_dec.replay()
+    if graphs is not None:
+        graphs[1].replay()
+        graphs[2].replay()
     else:
         marked_steps()
         decode_steps()
     torch.cuda.synchronize()
+    del graphs
 
     names = ["append", "q_absorb_plan", "attention", "merge_value_proj"]
     per = {n: [] for n in names}
@@ -384,20 +438,30 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     for evs in prof_ev:
         for j, n in enumerate(names):
             per[n].append(evs[j].elapsed_time(evs[j + 1]))
-    total_ms = max_over_ranks(sum(steps_ms), world, dev)
-    ms_per_step = total_ms / K
-    value = job_rate(work["units"], ms_per_step, world)
+    ms_per_step = max_over_ranks(sum(steps_ms), world, c.dev) / K
     kernel_ms = {n: statistics.fmean(v) for n, v in per.items()}
-    kernel_ms["marked_step"] = statistics.fmean(
-        evs[0].elapsed_time(evs[4]) for evs in prof_ev)
+    kernel_ms["marked_step"] = statistics.fmean(evs[0].elapsed_time(evs[4]) for evs in prof_ev)
     decode_ms = max_over_ranks(statistics.fmean(e[0].elapsed_time(e[1]) for e in dec_ev), world,
-                               dev)
+                               c.dev)
+    t_roof = decode_roofline_ms(c.work)
+    decode_only = {"value": job_rate(c.work["units"], decode_ms, world), "unit": UNIT,
+                   "ms_per_step": decode_ms, "roofline_frac": t_roof / decode_ms,
+                   "roofline_ms": t_roof,
+                   "what": "mla_decode alone (query absorption + planner, attention, merge + "
+                           "value projection), same L2 flush, graph-timed"}
+    return dict(ms_per_step=ms_per_step, value=job_rate(c.work["units"], ms_per_step, world),
+                kernel_ms=kernel_ms, decode_only=decode_only, clocks=clk, wall=t_wall,
+                roofline=attn_roofline(c.w, c.work, kernel_ms["attention"] / 1e3, ms_per_step))
 
-    # ---- e2e through the plain API from pinned host memory. Each step copies its inputs in and
-    # its output back inside the timed region: the append's inputs (x, seq_idx, pos) in one copy
-    # on the step's stream, the decode's (q, seq_lens) in one copy on a second stream that runs
-    # while the append kernels do (mla_decode waits for it), and the output in one copy; the
-    # host waits for the output.
+
+def measure_e2e(c: DeviceCase, flush_l2: L2Flush, K: int, world: int) -> dict:
+    """The same step through the plain API from pinned host memory: every step copies its
+    inputs in and its output back inside the timed region. The append's inputs (x, seq_idx,
+    pos) go in one copy on the step's stream, the decode's (q, seq_lens) in one copy on a
+    second stream that runs while the append kernels do (mla_decode waits for it), the output
+    in one copy that the host waits for."""
+    mla, dev = c.mla, c.dev
+
     def staged(parts):
         offs, off = [], 0
         for t in parts:
@@ -413,16 +477,17 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         return host, devb, views
 
     app_h, app_d, (x_e, si_e, pos_e) = staged(
-        [x_new_h.contiguous(), seq_idx_h.contiguous(), pos_h.contiguous()])
-    dec_h, dec_d, (q_e, lens_e) = staged([q_h.contiguous(), lens.contiguous()])
-    out_pin = torch.empty(out.shape, dtype=dt).pin_memory()
+        [c.x_new_h.contiguous(), c.seq_idx_h.contiguous(), c.pos_h.contiguous()])
+    dec_h, dec_d, (q_e, lens_e) = staged([c.q_h.contiguous(), c.lens.contiguous()])
+    out_pin = torch.empty(c.out.shape, dtype=c.out.dtype).pin_memory()
     h2d = app_h.numel() + dec_h.numel()
     d2h = out_pin.numel() * out_pin.element_size()
     main_s = torch.cuda.current_stream(dev)
     side_s = torch.cuda.Stream(device=dev)
     q_ready = torch.cuda.Event()
     K2 = min(K, 50)
-    e2e_ev = [(ev(), ev()) for _ in range(K2)]
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K2)]
     e2e_ms = []
     for i in range(K2):
         flush_l2(i)
@@ -433,10 +498,10 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             dec_d.copy_(dec_h, non_blocking=True)
             q_ready.record(side_s)
         app_d.copy_(app_h, non_blocking=True)
-        mla.mla_append_latent(cfg, x_e, w_dkv, kv_gain, si_e, pos_e, bt, cache, ws_a)
+        mla.mla_append_latent(c.cfg, x_e, c.w_dkv, c.kv_gain, si_e, pos_e, c.bt, c.cache, c.ws_a)
         main_s.wait_event(q_ready)
-        mla.mla_decode(cfg, q_e, cache, bt, lens_e, w_uk_t, w_uv, ws_d, out)
-        out_pin.copy_(out, non_blocking=True)
+        mla.mla_decode(c.cfg, q_e, c.cache, c.bt, lens_e, c.w_uk_t, c.w_uv, c.ws_d, c.out)
+        out_pin.copy_(c.out, non_blocking=True)
         b.record()
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
@@ -444,84 +509,95 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     err = mla.mla_get_device_error()
     if err != 0:
         raise RuntimeError(f"device error in the e2e loop: {mla.mla_status_string(err)}")
+    return {"value": job_rate(c.work["units"], e2e_step, world), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step}
 
-    # ---- roofline of the dominant kernel (latent attention)
-    pk, pk_kind = peaks()
-    t_attn = kernel_ms["attention"] / 1e3
-    hbm_peak = float(pk["hbm_gbs"])
-    tc_peak = float(pk["bf16_tflops"])
-    t_mem = work["cache_bytes"] / (hbm_peak * 1e9)
-    t_tc = work["attn_flops"] / (tc_peak * 1e12)
-    bound = "hbm" if t_mem >= t_tc else "tensor"
-    traffic = None
-    if os.path.exists(ATTN_PROFILE):
-        with open(ATTN_PROFILE) as f:
-            prof = json.load(f)
-        if prof.get("workload") == w.name and prof.get("kernel_source_sha") == kernel_sha():
-            traffic = prof.get("dram_bytes_per_launch")
-    if bound == "hbm":
-        roof = {"bound": "hbm", "achieved": work["cache_bytes"] / t_attn / 1e9, "peak": hbm_peak,
-                "unit": "GB/s"}
-    else:
-        roof = {"bound": "tensor", "achieved": work["attn_flops"] / t_attn / 1e12,
-                "peak": tc_peak, "unit": "TFLOP/s"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = traffic
-    roof["peak_source"] = f"{pk_kind} (MEASURED_PEAKS.json)" if pk_kind == "measured" else "fallback"
-    roof["kernel"] = "mla_decode_attn_kernel"
-    roof["algorithmic_bytes_per_launch"] = work["cache_bytes"]
-    roof["algorithmic_flops_per_launch"] = work["attn_flops"]
-    roof["tensor_achieved_tflops"] = work["attn_flops"] / t_attn / 1e12
-    roof["step_roofline_frac"] = max(
-        (work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
-        (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12)) / (ms_per_step / 1e3)
 
-    # mla_decode alone against the path's roofline: the larger of (cache + W_UK + W_UV bytes)
-    # over HBM bandwidth and (attention + projection FLOPs) over the tensor peak
-    t_roof = max((work["cache_bytes"] + work["weight_bytes"]) / (hbm_peak * 1e9),
-                 (work["attn_flops"] + work["proj_flops"]) / (tc_peak * 1e12))
-    decode_only = {"value": job_rate(work["units"], decode_ms, world), "unit": UNIT,
-                   "ms_per_step": decode_ms, "roofline_frac": t_roof / (decode_ms / 1e3),
-                   "roofline_ms": t_roof * 1e3,
-                   "what": "mla_decode alone (query absorption + planner, attention, merge + "
-                           "value projection), same L2 flush, graph-timed"}
+def run_ours(args, rank: int, world: int, local_rank: int):
+    import head_latent_attention_05_b200 as mla
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    w = WL.WORKLOADS[args.workload]
+    K, Wm = args.steps, max(3, args.warmup)
+    flush_l2 = L2Flush(dev)
+    c = DeviceCase(mla, w, dev)
+    m = measure_device(c, flush_l2, K, Wm, world, not args.no_graph, local_rank)
+    e2e = measure_e2e(c, flush_l2, K, world)
+    work = c.work
 
     line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": Wm, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "metric": METRIC, "value": m["value"], "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": m["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
         "config": {"workload": w.name, "batch_per_gpu": w.B, "global_batch": w.B * world,
                    "heads": w.H, "tq": w.Tq, "context": list(w.lens),
                    "cache_tokens_per_gpu": work["tokens"], "parallelism": f"dp{world}",
                    "l2": "flushed before every step, outside the step events: 256 MiB write, then a "
                          "256 MiB read that drains the written lines",
-                   "timing": ("CUDA graph of the K steps" if graph is not None else "eager")
+                   "timing": ("CUDA graph of the K steps" if not args.no_graph else "eager")
                    + "; kernel_ms and the roofline's kernel time from a second replay of the same"
                    " steps with event marks between the kernels",
                    "step": "mla_append_latent + mla_decode"},
-        "roofline": roof,
-        "kernel_ms": kernel_ms,
-        "decode_only": decode_only,
-        "e2e": {"value": job_rate(work["units"], e2e_step, world), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_step},
+        "roofline": m["roofline"],
+        "kernel_ms": m["kernel_ms"],
+        "decode_only": m["decode_only"],
+        "e2e": e2e,
         "gpu_launches": K * 5,
-        "clocks": clk,
-        "wall_s_timed_region": t_wall,
+        "clocks": m["clocks"],
+        "wall_s_timed_region": m["wall"],
     }
+    cpu_case = (c.lens, c.pt, c.weights, c.cache_host, c.x_new_h, c.pos_h, c.q_h)
+    del c
+
+    # the other bench-relevant workloads: the batch-16 x 4096 V2 shape and the tensor-bound
+    # long-context case, each with its own attention roofline (fewer steps)
+    if not args.no_extra:
+        extra = {}
+        for name in EXTRA_WORKLOADS:
+            if name == w.name:
+                continue
+            ce = DeviceCase(mla, WL.WORKLOADS[name], dev)
+            me = measure_device(ce, flush_l2, min(K, args.extra_steps), Wm, world,
+                                not args.no_graph, local_rank)
+            extra[name] = {"value": me["value"], "unit": UNIT, "ms_per_step": me["ms_per_step"],
+                           "steps": min(K, args.extra_steps), "roofline": me["roofline"],
+                           "kernel_ms": me["kernel_ms"], "decode_only": me["decode_only"],
+                           "clocks": me["clocks"], "gpu_launches": min(K, args.extra_steps) * 5}
+            del ce
+            torch.cuda.empty_cache()
+        line["other_workloads"] = extra
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        lens, pt, weights, cache_host, x_new_h, pos_h, q_h = cpu_case
+        threading = ("serial loop over (sequence, head) units; cores = the BLAS thread count that "
+                     "numpy's matrix products may use inside one unit")
         rate, units, desc = oracle_sample(w, lens, pt, weights, cache_host, x_new_h, pos_h, q_h,
                                           args.cpu_seconds)
         line["cpu_baseline"] = {"value": rate, "unit": UNIT, "cores": cpu_threads(),
-                                "kind": "oracle", "sample": desc}
+                                "kind": "oracle", "sample": desc, "threading": threading}
         # the same oracle's absorbed (latent-space) form, a second CPU number
         rate_a, _, desc_a = oracle_sample(w, lens, pt, weights, cache_host, x_new_h, pos_h, q_h,
                                           args.cpu_seconds / 3, form="absorbed")
         line["cpu_baseline_absorbed"] = {"value": rate_a, "unit": UNIT, "cores": cpu_threads(),
-                                         "kind": "oracle", "sample": desc_a}
+                                         "kind": "oracle", "sample": desc_a,
+                                         "threading": threading}
     if rank == 0:
         print(json.dumps(line), flush=True)
-    del graph, graph_prof, graph_dec
+
+
+def stored_traffic(workload: str):
+    """DRAM bytes per launch of the attention kernel from the committed ncu capture of this
+    workload, while the kernel's code still matches the one measured; else None."""
+    if not os.path.exists(ATTN_PROFILE):
+        return None
+    with open(ATTN_PROFILE) as f:
+        prof = json.load(f)
+    sha = kernel_sha()
+    for e in prof.get("captures", []):
+        if e.get("workload") == workload and e.get("kernel_source_sha") == sha:
+            return e.get("dram_bytes_per_launch")
+    return None
 
 
 def kernel_sha() -> str:

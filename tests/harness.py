@@ -113,3 +113,44 @@ def oracle_out(c: Case, b: int, heads, new_rows: np.ndarray) -> np.ndarray:
     W_UK, W_UV = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
     rows = oracle_rows_of(c, b, new_rows)
     return O.decode_expanded(c.q[b], rows, W_UK, W_UV, w.scale, w.rope_theta, heads=heads)
+
+
+def plant_score_staircase(c: Case, b: int, h: int, t: int = 0, base: float = 8.0,
+                          step: float = 7.0, period: int = 4, slot: int = 10) -> list:
+    """Overwrite one history row per 64-token page of sequence b so that, for head h and query
+    token t, the planted rows score base + step * (page % period) (natural-log units, after the
+    softmax scale) and dominate their page. Consecutive pages then raise the running maximum by
+    `step` > 8 ln 2, which is what makes the attention kernel move its reference maximum and
+    rescale its accumulator inside a segment. The planted row is c = (s / scale) q_lat / |q_lat|^2
+    with k_R = 0 (q_lat = q_nope W_UK[h], from the same inputs the oracle gets), rounded to the
+    cache dtype; host and device caches are updated alike. Returns the planted positions."""
+    w = c.w
+    L = int(c.lens[b])
+    W_UK, _ = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
+    q_lat = O.f64(c.q[b, t, h, :w.d_nope]) @ W_UK[h]
+    planted = []
+    for page_i in range((L - w.Tq) // W.PAGE_SIZE + 1):
+        j = page_i * W.PAGE_SIZE + slot
+        if j >= L - w.Tq:
+            break
+        s = base + step * (page_i % period)
+        row = np.zeros(w.row)
+        row[:w.d_c] = (s / w.scale) * q_lat / float(q_lat @ q_lat)
+        page = int(c.pt.block_table[b, page_i])
+        val = torch.from_numpy(row).to(w.torch_dtype)
+        c.cache_host[page, slot] = val
+        c.d["cache"][page, slot] = val.to(c.d["cache"].device)
+        planted.append(j)
+    return planted
+
+
+def oracle_scores(c: Case, b: int, h: int, t: int, rows: np.ndarray) -> np.ndarray:
+    """Scaled scores of head h, query token t of sequence b against every row (fp64, from the
+    oracle's own pieces), used to check properties of a test's inputs."""
+    w = c.w
+    W_UK, _ = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
+    L = rows.shape[0]
+    q = O.f64(c.q[b, t, h])
+    qf = np.concatenate([q[:w.d_nope], O.rope(q[w.d_nope:], L - w.Tq + t, w.rope_theta)])
+    K = np.concatenate([rows[:, :w.d_c] @ W_UK[h].T, rows[:, w.d_c:]], axis=1)
+    return (K @ qf) * w.scale
