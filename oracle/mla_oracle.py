@@ -114,8 +114,24 @@ def _softmax(s: np.ndarray) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
+def _visible(L: int, Tq: int, window: int) -> np.ndarray:
+    """mask[t, j]: key j is visible to query token t (position p = L - Tq + t).
+
+    Causal rule (「淺析DeepSeek多頭潛在注意力機制（MLA）」: the new token attends to all earlier
+    tokens and itself) and, for window > 0, the sliding window of the Streaming-MLA variant
+    (「Multi-Head Latent Attention（MLA）原理与工程实践全解析」 §7 keeps only the latents of the most
+    recent 1024 tokens): read here as key j visible iff p - window < j <= p.
+    """
+    pos = L - Tq + np.arange(Tq)
+    j = np.arange(L)[None, :]
+    vis = j <= pos[:, None]
+    if window > 0:
+        vis &= j > pos[:, None] - window
+    return vis
+
+
 def decode_expanded(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None,
-                    return_probs: bool = False):
+                    return_probs: bool = False, window: int = 0):
     """Attention output of the Tq newest tokens of one sequence, un-absorbed form.
 
     q     [Tq, H, d_nope + d_r]  un-rotated queries of the new tokens
@@ -127,7 +143,8 @@ def decode_expanded(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None,
     every head], V = c·W_UVᵀ, q_full = [q_nope | RoPE(q_rope)], scores = q_full·Kᵀ·scale with
     scale = 1/sqrt(d_nope + d_r), softmax, then probs·V. Query t sits at position L - Tq + t
     and sees keys 0 .. L - Tq + t (causal rule and the 1×(N+1) decode step in
-    「淺析DeepSeek多頭潛在注意力機制（MLA）」).
+    「淺析DeepSeek多頭潛在注意力機制（MLA）」); with window > 0 only the last `window` of them
+    (_visible).
     """
     q, rows = f64(q), f64(rows)
     W_UK, W_UV = f64(W_UK), f64(W_UV)
@@ -144,14 +161,14 @@ def decode_expanded(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None,
         V = c @ W_UV[h].T                                         # [L, d_v]
         qf = np.concatenate([q[:, h, :d_nope], rope(q[:, h, d_nope:], pos, theta)], axis=1)
         s = (qf @ K.T) * scale                                    # [Tq, L]
-        s[np.arange(L)[None, :] > pos[:, None]] = -np.inf
+        s[~_visible(L, Tq, window)] = -np.inf
         P = _softmax(s)
         out[:, j] = P @ V
         probs[:, j] = P
     return (out, probs) if return_probs else out
 
 
-def decode_absorbed(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None):
+def decode_absorbed(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None, window: int = 0):
     """Same result as decode_expanded, in the absorbed (latent-space) form.
 
     q_lat = q_nope·W_UK, score_j = (q_lat·c_j + RoPE(q_rope)·k_R,j)·scale, o_lat = P·c,
@@ -172,10 +189,63 @@ def decode_absorbed(q, rows, W_UK, W_UV, scale: float, theta: float, heads=None)
         q_lat = q[:, h, :d_nope] @ W_UK[h]                        # [Tq, d_c]
         q_r = rope(q[:, h, d_nope:], pos, theta)
         s = (q_lat @ c.T + q_r @ kr.T) * scale
-        s[np.arange(L)[None, :] > pos[:, None]] = -np.inf
+        s[~_visible(L, Tq, window)] = -np.inf
         o_lat = _softmax(s) @ c
         out[:, j] = o_lat @ W_UV[h].T
     return out
+
+
+def latent_partial(q, rows, W_UK, scale: float, theta: float, kv_begin: int, kv_end: int,
+                   heads=None, window: int = 0):
+    """Attention of the Tq newest tokens of one sequence over the keys kv_begin <= j < kv_end
+    only, in latent space: returns o [Tq, len(heads), d_c] = sum_j P_j c_j with P the softmax over
+    those keys (O / l), and lse [Tq, len(heads)] = ln sum_j exp(s_j) (-inf, and o = 0, when the
+    range holds no key the query sees).
+
+    The pages are silent on splitting one sequence's keys: this is the plain reading of split
+    attention, the softmax restricted to a subset of keys plus the log of its normaliser, which
+    merge_partials turns back into the whole softmax. Scores as in decode_absorbed.
+    """
+    q, rows = f64(q), f64(rows)
+    W_UK = f64(W_UK)
+    Tq, H = q.shape[0], q.shape[1]
+    L = rows.shape[0]
+    d_nope, d_c = W_UK.shape[1], W_UK.shape[2]
+    heads = list(range(H)) if heads is None else list(heads)
+    c, kr = rows[:, :d_c], rows[:, d_c:]
+    pos = L - Tq + np.arange(Tq)
+    vis = _visible(L, Tq, window)
+    idx = np.arange(L)
+    vis &= (idx >= kv_begin)[None, :] & (idx < kv_end)[None, :]
+    o = np.zeros((Tq, len(heads), d_c))
+    lse = np.full((Tq, len(heads)), -np.inf)
+    for jh, h in enumerate(heads):
+        q_lat = q[:, h, :d_nope] @ W_UK[h]
+        q_r = rope(q[:, h, d_nope:], pos, theta)
+        s = (q_lat @ c.T + q_r @ kr.T) * scale
+        for t in range(Tq):
+            st = s[t, vis[t]]
+            if st.size == 0:
+                continue
+            m = st.max()
+            e = np.exp(st - m)
+            o[t, jh] = (e / e.sum()) @ c[vis[t]]
+            lse[t, jh] = m + np.log(e.sum())
+    return o, lse
+
+
+def merge_partials(o_parts, lse_parts):
+    """Merge partial results over disjoint key ranges: sum_k e^(lse_k - M) o_k / sum_k
+    e^(lse_k - M), M = max_k lse_k (zeros where every lse is -inf). o_parts [K, ..., d],
+    lse_parts [K, ...]. Because e^(lse_k) is the normaliser of part k, this is the softmax over
+    the union of the ranges applied to the same values."""
+    o_parts, lse_parts = f64(o_parts), f64(lse_parts)
+    M = lse_parts.max(axis=0)
+    Ms = np.where(np.isfinite(M), M, 0.0)
+    w = np.where(np.isfinite(lse_parts), np.exp(lse_parts - Ms[None]), 0.0)
+    den = w.sum(axis=0)
+    num = (w[..., None] * o_parts).sum(axis=0)
+    return np.where(den[..., None] > 0, num / np.where(den > 0, den, 1.0)[..., None], 0.0)
 
 
 def module_attention(x, w_dkv, kv_gain, wkv_b, w_qa, q_gain, w_qb, H, d_c, d_r, d_nope, d_v,

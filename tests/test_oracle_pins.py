@@ -411,3 +411,78 @@ def test_query_path_brute_force():
     q = [sum(W["w_qb"][o, i] * qn[i] for i in range(q_lora)) for o in range(H * (d_nope + d_r))]
     got = O.query_from_x(x, W["w_qa"], W["q_gain"], W["w_qb"], H, d_nope, d_r, eps)
     np.testing.assert_allclose(got, np.array(q).reshape(H, d_nope + d_r), rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------ sliding window and key ranges
+
+def test_window_special_cases():
+    """window >= L is plain causal attention; window = 1 returns each query's own value."""
+    rng = np.random.default_rng(30)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=40, Tq=3)
+    full = O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0)
+    np.testing.assert_array_equal(O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0,
+                                                    window=40), full)
+    own = O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0, window=1)
+    for t in range(3):
+        expect = np.einsum("d,hvd->hv", rows[37 + t, :16], W_UV)
+        np.testing.assert_allclose(own[t], expect, rtol=1e-13, atol=1e-13)
+
+
+def test_window_equals_truncated_history():
+    """With window W, the output equals plain attention over the last W rows only, with the
+    query's position (and RoPE angle) unchanged: brute force by cutting the history. RoPE depends
+    only on relative positions, so the cut is rotated back to position 0 and the query too."""
+    rng = np.random.default_rng(31)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=50, Tq=1)
+    W = 13
+    got = O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0, window=W)
+    # keep the last W rows; re-rotate their k_R by -(50 - W) and the query's q_rope by the same
+    tail = rows[50 - W:].copy()
+    tail[:, 16:] = O.rope(tail[:, 16:], -(50 - W), 10000.0)
+    ref = O.decode_expanded(q, tail, W_UK, W_UV, 0.3, 10000.0)
+    np.testing.assert_allclose(got, ref, rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("window", [0, 7])
+def test_absorbed_equals_expanded_with_window(window):
+    rng = np.random.default_rng(32)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=30, Tq=2)
+    a = O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0, window=window)
+    b = O.decode_absorbed(q, rows, W_UK, W_UV, 0.3, 10000.0, window=window)
+    assert np.max(np.abs(a - b)) <= 1e-12 * np.max(np.abs(a))
+
+
+@pytest.mark.parametrize("cuts,window", [([0, 64, 100], 0), ([0, 1, 2, 100], 0),
+                                         ([0, 50, 100], 30), ([0, 99, 100], 0)])
+def test_partials_merge_to_the_whole_softmax(cuts, window):
+    """Splitting the keys at any cut points and merging the partials reproduces the absorbed
+    form's latent output over all keys (then W_UV gives decode_expanded's output)."""
+    rng = np.random.default_rng(33)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=100, Tq=2)
+    parts = [O.latent_partial(q, rows, W_UK, 0.3, 10000.0, a, b, window=window)
+             for a, b in zip(cuts[:-1], cuts[1:])]
+    o = O.merge_partials(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]))
+    out = np.einsum("thd,hvd->thv", o, W_UV)
+    ref = O.decode_expanded(q, rows, W_UK, W_UV, 0.3, 10000.0, window=window)
+    np.testing.assert_allclose(out, ref, rtol=1e-11, atol=1e-12)
+
+
+def test_partial_of_an_empty_range_is_minus_infinity_and_ignored():
+    rng = np.random.default_rng(34)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=20, Tq=1)
+    o, lse = O.latent_partial(q, rows, W_UK, 0.3, 10000.0, 20, 20)
+    assert np.all(lse == -np.inf) and np.all(o == 0.0)
+    o2, lse2 = O.latent_partial(q, rows, W_UK, 0.3, 10000.0, 0, 20)
+    m = O.merge_partials(np.stack([o, o2]), np.stack([lse, lse2]))
+    np.testing.assert_array_equal(m, o2)
+
+
+def test_partial_lse_is_the_log_normaliser():
+    """Brute force: lse = ln sum_j exp(s_j) over the range, s_j from the expanded form's keys."""
+    rng = np.random.default_rng(35)
+    q, rows, W_UK, W_UV = _rand_decode(rng, L=12, Tq=1)
+    _, lse = O.latent_partial(q, rows, W_UK, 0.3, 10000.0, 3, 9, heads=[1])
+    K = np.concatenate([rows[:, :16] @ W_UK[1].T, rows[:, 16:]], axis=1)
+    qf = np.concatenate([q[0, 1, :8], O.rope(q[0, 1, 8:], 11, 10000.0)])
+    s = [0.3 * sum(qf[i] * K[j, i] for i in range(16)) for j in range(3, 9)]
+    assert abs(lse[0, 0] - math.log(sum(math.exp(v) for v in s))) <= 1e-12 * abs(lse[0, 0])
