@@ -31,7 +31,9 @@ EXPORTED = (
     "mla_status_string", "mla_absorb_weights", "mla_append_workspace_size", "mla_append_latent",
     "mla_decode_workspace_size", "mla_decode", "mla_decode_profiled", "mla_decode_noalloc",
     "mla_prefill_ref_workspace_size",
-    "mla_prefill_ref", "mla_get_device_error",
+    "mla_prefill_ref", "mla_get_device_error", "mla_query_workspace_size", "mla_query",
+    "mla_output_workspace_size", "mla_output", "mla_decode_partial", "mla_combine_workspace_size",
+    "mla_combine", "mla_prefill_workspace_size", "mla_prefill",
 )
 
 
@@ -47,18 +49,18 @@ class MlaConfig(ctypes.Structure):
         ("d_rope", ctypes.c_int32), ("d_nope", ctypes.c_int32), ("d_v", ctypes.c_int32),
         ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
-        ("rope_theta", ctypes.c_float),
+        ("rope_theta", ctypes.c_float), ("window", ctypes.c_int32),
     ]
 
 
 def make_config(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size=64, dtype="bf16",
-                softmax_scale=None, rms_eps=1e-6, rope_theta=10000.0) -> MlaConfig:
+                softmax_scale=None, rms_eps=1e-6, rope_theta=10000.0, window=0) -> MlaConfig:
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(d_nope + d_rope)
     dt = {"bf16": MLA_DTYPE_BF16, "f32": MLA_DTYPE_F32,
           torch.bfloat16: MLA_DTYPE_BF16, torch.float32: MLA_DTYPE_F32}[dtype]
     return MlaConfig(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size, dt,
-                     softmax_scale, rms_eps, rope_theta)
+                     softmax_scale, rms_eps, rope_theta, window)
 
 
 _lib = None
@@ -87,6 +89,17 @@ def load_library() -> ctypes.CDLL:
         "mla_prefill_ref_workspace_size": (SZ, [CFG, I32, I32]),
         "mla_prefill_ref": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ, P, P]),
         "mla_get_device_error": (ctypes.c_int, [P]),
+        "mla_query_workspace_size": (SZ, [CFG, I32, I32]),
+        "mla_query": (ctypes.c_int, [CFG, I32, P, I32, P, P, P, P, SZ, P, P]),
+        "mla_output_workspace_size": (SZ, [CFG, I32]),
+        "mla_output": (ctypes.c_int, [CFG, P, I32, P, P, SZ, P, P]),
+        "mla_decode_partial": (ctypes.c_int, [CFG, P, I32, I32, P, I32, P, I32, P, P, P, P, P, SZ,
+                                              P, P, P]),
+        "mla_combine_workspace_size": (SZ, [CFG, I32, I32]),
+        "mla_combine": (ctypes.c_int, [CFG, I32, I32, I32, P, P, P, P, SZ, P, P]),
+        "mla_prefill_workspace_size": (SZ, [CFG, I32, I32]),
+        "mla_prefill": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ,
+                                       P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -194,6 +207,72 @@ def mla_prefill_ref(cfg: MlaConfig, x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens
         _ptr(cache), cache.shape[0], _ptr(workspace),
         workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)),
         "mla_prefill_ref")
+
+
+def mla_query_workspace_size(cfg: MlaConfig, q_lora: int, n_tok: int) -> int:
+    return int(load_library().mla_query_workspace_size(ctypes.byref(cfg), q_lora, n_tok))
+
+
+def mla_query(cfg: MlaConfig, x, w_qa, q_gain, w_qb, workspace, q_out, stream=None):
+    """q path: q_out [n_tok, H, d_nope + d_rope] from hidden states x [n_tok, d_model]."""
+    n_tok, q_lora = x.shape[0], w_qa.shape[0]
+    _check(load_library().mla_query(
+        ctypes.byref(cfg), q_lora, _ptr(x), n_tok, _ptr(w_qa), _ptr(q_gain), _ptr(w_qb),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(q_out),
+        _stream(stream)), "mla_query")
+
+
+def mla_output_workspace_size(cfg: MlaConfig, n_tok: int) -> int:
+    return int(load_library().mla_output_workspace_size(ctypes.byref(cfg), n_tok))
+
+
+def mla_output(cfg: MlaConfig, attn, w_o, workspace, y, stream=None):
+    """Output projection: y [n_tok, d_model] from attention outputs attn [n_tok, H, d_v]."""
+    _check(load_library().mla_output(
+        ctypes.byref(cfg), _ptr(attn), attn.shape[0], _ptr(w_o), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(y), _stream(stream)), "mla_output")
+
+
+def mla_decode_partial(cfg: MlaConfig, q, cache, block_table, seq_lens, kv_begin, kv_end, w_uk_t,
+                       workspace, o_part, lse, stream=None):
+    """Decode over keys kv_begin[b] <= j < kv_end[b] only: o_part [B*Tq*H, d_c] (O / l) and
+    lse [B*Tq*H] (natural log), to be merged with other ranges' partials by mla_combine."""
+    batch, tq = q.shape[0], q.shape[1]
+    _check(load_library().mla_decode_partial(
+        ctypes.byref(cfg), _ptr(q), batch, tq, _ptr(cache), cache.shape[0], _ptr(block_table),
+        block_table.shape[1], _ptr(seq_lens), _ptr(kv_begin), _ptr(kv_end), _ptr(w_uk_t),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _ptr(o_part), _ptr(lse),
+        _stream(stream)), "mla_decode_partial")
+
+
+def mla_combine_workspace_size(cfg: MlaConfig, batch: int, tq: int) -> int:
+    return int(load_library().mla_combine_workspace_size(ctypes.byref(cfg), batch, tq))
+
+
+def mla_combine(cfg: MlaConfig, o_parts, lse_parts, w_uv, workspace, out, stream=None):
+    """Merge n_parts partials (o_parts [n_parts, B*Tq*H, d_c], lse_parts [n_parts, B*Tq*H]) and
+    project into out [B, Tq, H, d_v]."""
+    n_parts, batch, tq = o_parts.shape[0], out.shape[0], out.shape[1]
+    ws = workspace if workspace is not None else torch.empty(0, dtype=torch.uint8)
+    _check(load_library().mla_combine(
+        ctypes.byref(cfg), n_parts, batch, tq, _ptr(o_parts), _ptr(lse_parts), _ptr(w_uv),
+        ctypes.c_void_p(ws.data_ptr()) if ws.numel() else None, ws.numel() * ws.element_size(),
+        _ptr(out), _stream(stream)), "mla_combine")
+
+
+def mla_prefill_workspace_size(cfg: MlaConfig, batch: int, t_new: int) -> int:
+    return int(load_library().mla_prefill_workspace_size(ctypes.byref(cfg), batch, t_new))
+
+
+def mla_prefill(cfg: MlaConfig, x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens, block_table, cache,
+                workspace, out, stream=None):
+    """Tensor-core prefill: same arguments and results as mla_prefill_ref."""
+    batch, t_new = q.shape[0], q.shape[1]
+    _check(load_library().mla_prefill(
+        ctypes.byref(cfg), _ptr(x), _ptr(q), batch, t_new, _ptr(w_dkv), _ptr(kv_gain),
+        _ptr(w_uk_t), _ptr(w_uv), _ptr(seq_lens), _ptr(block_table), block_table.shape[1],
+        _ptr(cache), cache.shape[0], _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _ptr(out), _stream(stream)), "mla_prefill")
 
 
 def mla_get_device_error(stream=None) -> int:

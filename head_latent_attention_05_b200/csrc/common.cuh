@@ -79,6 +79,30 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
+// Which cached keys a query may attend to. Query token t of a sequence of length L with Tq new
+// tokens sits at position p = L - Tq + t and sees the keys j with lo <= j <= hi:
+//   causal          j <= p (a query sees itself and earlier tokens),
+//   sliding window  j > p - window when window > 0 (only the last `window` tokens are kept),
+//   key range       kv_begin[b] <= j < kv_end[b] when given (the share of a sequence's keys that
+//                   one GPU holds when a long context is split over several GPUs).
+// lo > hi means the query sees no key here.
+struct KeyRange {
+  const int32_t* kv_begin;   // [B] or null (= 0)
+  const int32_t* kv_end;     // [B] or null (= L)
+  int window;                // 0 = unlimited
+};
+
+__device__ __forceinline__ void visible_keys(const KeyRange& kr, int b, int L, int Tq, int t,
+                                             int* lo, int* hi) {
+  const int p = L - Tq + t;
+  int l = 0, h = p;
+  if (kr.window > 0) l = max(l, p - kr.window + 1);
+  if (kr.kv_begin != nullptr) l = max(l, kr.kv_begin[b]);
+  if (kr.kv_end != nullptr) h = min(h, kr.kv_end[b] - 1);
+  *lo = l;
+  *hi = h;
+}
+
 constexpr int MLA_MAX_ROPE_PAIRS = 64;   // d_rope <= 128
 
 // Per rotary pair i, f_i = theta^(-2i/d_rope) / pi split into two floats (f_hi + f_lo carries

@@ -53,6 +53,7 @@ mla_status check_config(const mla_config* c) {
   if (c->dtype != MLA_DTYPE_F32 && c->dtype != MLA_DTYPE_BF16) return MLA_ERR_INVALID_ARG;
   if (!(c->softmax_scale > 0.0f) || !std::isfinite(c->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.0f) || !(c->rope_theta > 0.0f)) return MLA_ERR_INVALID_ARG;
+  if (c->window < 0) return MLA_ERR_INVALID_ARG;
   // every row must stay 16-byte aligned for vector loads and TMA
   const int64_t row_bytes = static_cast<int64_t>(c->d_c + c->d_rope) * elem_bytes(c);
   if (row_bytes % 16 != 0) return MLA_ERR_UNSUPPORTED;
@@ -314,7 +315,7 @@ bool tc_append_shape(const mla_config* c) {
 
 struct DecodeLayout {
   int P, n_mt, R, U, max_segs;
-  int32_t *unit_tiles, *unit_seg, *pair_seg;
+  int32_t *unit_first, *unit_tiles, *unit_seg, *pair_seg;
   AttnSeg* segs;
   __nv_bfloat16* qhat;
   __nv_bfloat16* o_part;
@@ -338,6 +339,7 @@ DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
   L.U = B * L.n_mt;
   L.max_segs = L.U + L.P;
   Carve cv(ws);
+  L.unit_first = cv.take<int32_t>(L.U);
   L.unit_tiles = cv.take<int32_t>(L.U);
   L.unit_seg = cv.take<int32_t>(L.U + 1);
   L.pair_seg = cv.take<int32_t>(L.P + 1);
@@ -369,12 +371,15 @@ SimtLayout simt_layout(const mla_config* c, int64_t rows, int64_t n_append_tok, 
 
 // -------------------------------------------------------------------- SIMT decode (any T)
 
+// keys: which keys each row sees; with o_lat_out given the latent output (O / l) goes there
+// with its log-sum-exp in lse_out, and the value projection is skipped.
 template <typename T>
 mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const void* cache,
                        int num_pages, const int32_t* block_table, int max_pages,
                        const int32_t* seq_lens, const void* w_uk_t, const void* w_uv,
                        const SimtLayout& L, void* out, cudaStream_t st,
-                       void* const* events = nullptr) {
+                       void* const* events = nullptr, KeyRange keys = KeyRange{nullptr, nullptr, 0},
+                       float* o_lat_out = nullptr, float* lse_out = nullptr) {
   auto mark = [&](int i) {
     if (events != nullptr && events[i] != nullptr)
       record_mark(static_cast<cudaEvent_t>(events[i]), st);
@@ -382,6 +387,7 @@ mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const 
   const int rows = B * Tq * c->n_heads;
   const int row = c->d_c + c->d_rope;
   const int max_pos = max_pages * c->page_size;
+  if (keys.window == 0) keys.window = c->window;
   qabs_simt_kernel<T><<<rows, 256, (c->d_nope + c->d_rope) * sizeof(float), st>>>(
       static_cast<const T*>(q), static_cast<const T*>(w_uk_t), seq_lens, L.qhat, c->n_heads,
       Tq, c->d_c, c->d_rope, c->d_nope, max_pos, rope_freqs(c));
@@ -389,9 +395,11 @@ mla_status simt_decode(const mla_config* c, const void* q, int B, int Tq, const 
   if (!allow_smem(attn_simt_kernel<T>, attn_smem)) return MLA_ERR_CUDA;
   mark(1);
   attn_simt_kernel<T><<<rows, 256, attn_smem, st>>>(
-      L.qhat, static_cast<const T*>(cache), block_table, seq_lens, L.o_lat, c->n_heads, Tq,
-      c->d_c, c->d_rope, max_pages, num_pages, c->page_size, c->softmax_scale);
+      L.qhat, static_cast<const T*>(cache), block_table, seq_lens,
+      o_lat_out != nullptr ? o_lat_out : L.o_lat, c->n_heads, Tq, c->d_c, c->d_rope, max_pages,
+      num_pages, c->page_size, c->softmax_scale, keys, lse_out);
   mark(2);
+  if (o_lat_out != nullptr) return last_launch_status();
   outproj_simt_kernel<T><<<rows, 256, c->d_c * sizeof(float), st>>>(
       L.o_lat, static_cast<const T*>(w_uv), static_cast<T*>(out), c->n_heads, c->d_c, c->d_v);
   return last_launch_status();
@@ -422,6 +430,141 @@ __global__ void prefill_positions_kernel(const int32_t* __restrict__ seq_lens, i
   const int b = i / t_new, t = i % t_new;
   seq_idx[i] = b;
   pos[i] = seq_lens[b] - t_new + t;  // out-of-range values are caught by the append kernel
+}
+
+// ------------------------------------------------------- q path and output projection plans
+
+// Split-K plan of a weight-streaming GEMM with m_tiles x n_tiles output tiles and k_chunks
+// 64-wide K chunks: enough K-splits that the grid covers about `ctas` CTAs (one per SM when
+// ctas is the SM count), every split non-empty.
+struct SplitPlan {
+  int k_chunks, chunks_per_split, k_splits;
+};
+SplitPlan split_plan(int m_tiles, int n_tiles, int k_chunks, int ctas, bool round_up) {
+  SplitPlan p{};
+  p.k_chunks = k_chunks;
+  const int tiles = m_tiles * n_tiles;
+  int splits = round_up ? (ctas + tiles - 1) / tiles : ctas / tiles;
+  splits = splits < 1 ? 1 : (splits > k_chunks ? k_chunks : splits);
+  p.chunks_per_split = (k_chunks + splits - 1) / splits;
+  p.k_splits = (k_chunks + p.chunks_per_split - 1) / p.chunks_per_split;
+  return p;
+}
+
+int sm_count_or_default() {
+  const int n = device_sm_count();
+  return n > 0 ? n : 148;
+}
+
+bool tc_query_shape(const mla_config* c, int q_lora) {
+  return c->dtype == MLA_DTYPE_BF16 && c->d_model % 64 == 0 && q_lora % 64 == 0;
+}
+bool tc_output_shape(const mla_config* c) {
+  return c->dtype == MLA_DTYPE_BF16 && (c->n_heads * c->d_v) % 64 == 0;
+}
+
+struct QueryPlan {
+  SplitPlan a;      // wq_a: M = q_lora, K = d_model
+  int bn, n_tiles, m_tiles_a, m_tiles_b, m_per_cta_b;
+};
+QueryPlan query_plan(const mla_config* c, int q_lora, int n_tok) {
+  QueryPlan p{};
+  p.bn = pick_bn(n_tok);
+  p.n_tiles = (n_tok + p.bn - 1) / p.bn;
+  p.m_tiles_a = (q_lora + 127) / 128;
+  p.a = split_plan(p.m_tiles_a, p.n_tiles, c->d_model / 64, sm_count_or_default(), true);
+  const int M_b = c->n_heads * (c->d_nope + c->d_rope);
+  p.m_tiles_b = (M_b + 127) / 128;
+  // wq_b: consecutive m-tiles per CTA so that one wave of CTAs covers the weight
+  int per = (p.m_tiles_b * p.n_tiles + sm_count_or_default() - 1) / sm_count_or_default();
+  while (per > 1 && p.bn * per > 512) --per;   // the accumulators must fit TMEM
+  p.m_per_cta_b = per < 1 ? 1 : per;
+  return p;
+}
+
+struct QueryLayout {
+  float* partial;   // [splits][n_tok][q_lora] (tensor-core path) or [n_tok][q_lora] (SIMT)
+  void* qa;         // [n_tok][q_lora] in cfg->dtype
+  float* q32;       // [n_tok][M_b] fp32 (SIMT path only)
+  size_t bytes;
+};
+QueryLayout query_layout(const mla_config* c, int q_lora, int n_tok, void* ws) {
+  QueryLayout L{};
+  Carve cv(ws);
+  const size_t M_b = static_cast<size_t>(c->n_heads) * (c->d_nope + c->d_rope);
+  if (tc_query_shape(c, q_lora)) {
+    const QueryPlan p = query_plan(c, q_lora, n_tok);
+    L.partial = cv.take<float>(static_cast<size_t>(p.a.k_splits) * n_tok * q_lora);
+    L.qa = cv.take<__nv_bfloat16>(static_cast<size_t>(n_tok) * q_lora);
+  } else {
+    L.partial = cv.take<float>(static_cast<size_t>(n_tok) * q_lora);
+    L.qa = cv.take<float>(static_cast<size_t>(n_tok) * q_lora);   // room for either dtype
+    L.q32 = cv.take<float>(static_cast<size_t>(n_tok) * M_b);
+  }
+  L.bytes = cv.off;
+  return L;
+}
+
+struct OutputPlan {
+  SplitPlan s;
+  int bn, n_tiles, m_tiles;
+};
+OutputPlan output_plan(const mla_config* c, int n_tok) {
+  OutputPlan p{};
+  p.bn = pick_bn(n_tok);
+  p.n_tiles = (n_tok + p.bn - 1) / p.bn;
+  p.m_tiles = (c->d_model + 127) / 128;
+  // as many K-splits as keep the grid within one wave of CTAs
+  p.s = split_plan(p.m_tiles, p.n_tiles, c->n_heads * c->d_v / 64, sm_count_or_default(), false);
+  return p;
+}
+size_t output_ws_bytes(const mla_config* c, int n_tok) {
+  const size_t per = static_cast<size_t>(n_tok) * c->d_model;
+  if (tc_output_shape(c)) return align_up(static_cast<size_t>(output_plan(c, n_tok).s.k_splits) * per * sizeof(float));
+  return align_up(per * sizeof(float));
+}
+
+// Launch a bf16 tensor-core GEMM D = W · Xᵀ: W [M, K] weights (K contiguous), X [N, K]
+// activations, epilogue epi; m_per_cta consecutive m-tiles per CTA, K split as in sp.
+template <class Epi>
+mla_status weight_gemm(const void* w, int M, int K, const void* x, int N, const SplitPlan& sp,
+                       int m_per_cta, int bn, const Epi& epi, cudaStream_t st) {
+  CUtensorMap mA, mB;
+  const uint64_t da[3] = {static_cast<uint64_t>(K), static_cast<uint64_t>(M), 1};
+  const uint64_t sa[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * 2 * M};
+  const uint32_t ba[3] = {64, 128, 1};
+  const uint64_t db[3] = {static_cast<uint64_t>(K), 1, static_cast<uint64_t>(N)};
+  const uint64_t sb[2] = {static_cast<uint64_t>(K) * 2, static_cast<uint64_t>(K) * 2};
+  const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(bn)};
+  if (!make_map(&mA, w, 3, da, sa, ba) || !make_map(&mB, x, 3, db, sb, bb)) return MLA_ERR_CUDA;
+  GemmShape shp{M, N, sp.k_chunks, sp.chunks_per_split, sp.k_splits, 0, m_per_cta, 0};
+  return launch_gemm(mA, mB, shp, (M + 127) / 128, 1, epi, st, bn);
+}
+
+// The split merge fused with the value projection (vproj_merge_kernel) over the rows of p;
+// pdl: launched with programmatic dependent launch (it follows the library's own kernel).
+mla_status launch_vproj(const mla_config* cfg, const void* w_uv, const VprojParams& vp,
+                        cudaStream_t st, bool pdl) {
+  CUtensorMap mA;
+  const int H = cfg->n_heads;
+  const uint64_t da[3] = {ATT_DC, static_cast<uint64_t>(cfg->d_v), static_cast<uint64_t>(H)};
+  const uint64_t sa[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * cfg->d_v};
+  const uint32_t ba[3] = {64, 128, 1};
+  if (!make_map(&mA, w_uv, 3, da, sa, ba)) return MLA_ERR_CUDA;
+  const int n_q = vp.n_q;
+  const int bn = pick_bn(n_q) > 64 ? 64 : pick_bn(n_q);
+  const dim3 grid((cfg->d_v + 127) / 128, (n_q + bn - 1) / bn, H);
+  auto go = [&](auto kern, int smem) -> mla_status {
+    if (!allow_smem(kern, smem)) return MLA_ERR_CUDA;
+    if (pdl) return launch_pdl(kern, grid, dim3(VP_THREADS), smem, st, mA, vp);
+    kern<<<grid, VP_THREADS, smem, st>>>(mA, vp);
+    return last_launch_status();
+  };
+  switch (bn) {
+    case 16: return go(vproj_merge_kernel<16>, vproj_smem_bytes<16>());
+    case 32: return go(vproj_merge_kernel<32>, vproj_smem_bytes<32>());
+    default: return go(vproj_merge_kernel<64>, vproj_smem_bytes<64>());
+  }
 }
 
 }  // namespace
@@ -538,17 +681,26 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t t
   return simt_layout(cfg, static_cast<int64_t>(batch) * tq * cfg->n_heads, 0, nullptr).bytes;
 }
 
+// mla_decode and its variants. kv_begin / kv_end (optional) restrict the keys read; with
+// part_out given the result is the merged latent output O / l of each row (and lse_out its
+// natural-log log-sum-exp) instead of the projected output, and w_uv / out are not used.
 static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
                               const void* cache, int32_t num_pages, const int32_t* block_table,
                               int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
                               const void* w_uv, void* workspace, size_t ws_bytes, void* out,
-                              void* stream, void* const* events) {
+                              void* stream, void* const* events,
+                              const int32_t* kv_begin = nullptr, const int32_t* kv_end = nullptr,
+                              void* part_out = nullptr, float* lse_out = nullptr) {
   const mla_status cs = check_config(cfg);
   if (cs != MLA_OK) return cs;
   if (batch < 1 || tq < 1 || num_pages < 1 || max_pages < 1) return MLA_ERR_INVALID_ARG;
-  const void* ptrs[] = {q, cache, block_table, seq_lens, w_uk_t, w_uv, workspace, out};
+  const bool partial = part_out != nullptr;
+  const void* ptrs[] = {q, cache, block_table, seq_lens, w_uk_t, workspace,
+                        partial ? part_out : out, partial ? static_cast<void*>(lse_out) : w_uv};
   for (const void* p : ptrs)
     if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if ((kv_begin == nullptr) != (kv_end == nullptr)) return MLA_ERR_INVALID_ARG;
+  const KeyRange keys{kv_begin, kv_end, cfg->window};
   if (static_cast<int64_t>(max_pages) * cfg->page_size > (1 << 30)) return MLA_ERR_INVALID_ARG;
   if (cfg->dtype == MLA_DTYPE_BF16 && !tc_decode_shape(cfg)) return MLA_ERR_UNSUPPORTED;
   if (ws_bytes < mla_decode_workspace_size(cfg, batch, tq)) return MLA_ERR_WORKSPACE_TOO_SMALL;
@@ -565,7 +717,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     mark(0);
     const mla_status s = simt_decode<float>(cfg, q, batch, tq, cache, num_pages, block_table,
                                             max_pages, seq_lens, w_uk_t, w_uv, L, out, st,
-                                            events);
+                                            events, keys, static_cast<float*>(part_out), lse_out);
     mark(3);
     return s;
   }
@@ -597,8 +749,8 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
       return MLA_ERR_CUDA;
     const int m_per_cta = ATT_DC / 128;
     GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1, m_per_cta, 1};
-    PlanParams pp{seq_lens, batch, tq, L.n_mt, max_pos, L.P, L.max_segs,
-                  L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
+    PlanParams pp{seq_lens, batch, tq, H, L.n_mt, max_pos, L.P, L.max_segs, keys,
+                  L.unit_first, L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
     EpiQhat epi{L.qhat, static_cast<const __nv_bfloat16*>(q), seq_lens, H, tq, ATT_DC, ATT_DR,
                 cfg->d_nope, n_q, max_pos, bn, pp, rope_freqs(cfg)};
     const mla_status s = launch_gemm(mA, mB, shp, ATT_DC / 128, H, epi, st, bn);
@@ -622,7 +774,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
       return MLA_ERR_CUDA;
     AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
-                  cfg->softmax_scale * 1.4426950408889634f};
+                  cfg->softmax_scale * 1.4426950408889634f, keys};
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
     mark(1);
     const mla_status s = launch_pdl(mla_decode_attn_kernel, dim3(2 * L.P), dim3(ATT_THREADS),
@@ -630,42 +782,25 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     if (s != MLA_OK) return s;
   }
 
-  // (3) merge the split partials and project: out = o_lat · W_UVᵀ per head
-  {
-    CUtensorMap mA;
-    const uint64_t da[3] = {ATT_DC, static_cast<uint64_t>(cfg->d_v), static_cast<uint64_t>(H)};
-    const uint64_t sa[2] = {ATT_DC * 2, static_cast<uint64_t>(ATT_DC) * 2 * cfg->d_v};
-    const uint32_t ba[3] = {64, 128, 1};
-    if (!make_map(&mA, w_uv, 3, da, sa, ba)) return MLA_ERR_CUDA;
-    VprojParams vp{L.o_part, L.lse, L.unit_seg, static_cast<__nv_bfloat16*>(out), H, tq, L.n_mt,
-                   n_q, cfg->d_v};
-    const int bn = pick_bn(n_q) > 64 ? 64 : pick_bn(n_q);
-    const dim3 grid((cfg->d_v + 127) / 128, (n_q + bn - 1) / bn, H);
+  // (3a) partial decode: merge each row's segments into one partial and its lse
+  if (partial) {
     mark(2);
-    mla_status s;
-    switch (bn) {
-      case 16:
-        s = allow_smem(vproj_merge_kernel<16>, vproj_smem_bytes<16>())
-                ? launch_pdl(vproj_merge_kernel<16>, grid, dim3(VP_THREADS),
-                             vproj_smem_bytes<16>(), st, mA, vp)
-                : MLA_ERR_CUDA;
-        break;
-      case 32:
-        s = allow_smem(vproj_merge_kernel<32>, vproj_smem_bytes<32>())
-                ? launch_pdl(vproj_merge_kernel<32>, grid, dim3(VP_THREADS),
-                             vproj_smem_bytes<32>(), st, mA, vp)
-                : MLA_ERR_CUDA;
-        break;
-      default:
-        s = allow_smem(vproj_merge_kernel<64>, vproj_smem_bytes<64>())
-                ? launch_pdl(vproj_merge_kernel<64>, grid, dim3(VP_THREADS),
-                             vproj_smem_bytes<64>(), st, mA, vp)
-                : MLA_ERR_CUDA;
-        break;
-    }
+    const int rows = batch * L.R;
+    const mla_status s = launch_pdl(merge_partials_kernel, dim3((rows + 3) / 4), dim3(256), 0, st,
+                                    static_cast<const __nv_bfloat16*>(L.o_part),
+                                    static_cast<const float*>(L.lse),
+                                    static_cast<const int32_t*>(L.unit_seg), rows, L.R, L.n_mt,
+                                    static_cast<__nv_bfloat16*>(part_out), lse_out);
     mark(3);
     return s;
   }
+  // (3) merge the split partials and project: out = o_lat · W_UVᵀ per head
+  VprojParams vp{L.o_part, L.lse, L.unit_seg, static_cast<__nv_bfloat16*>(out), H, tq, L.n_mt,
+                 n_q, cfg->d_v, 0};
+  mark(2);
+  const mla_status s = launch_vproj(cfg, w_uv, vp, st, true);
+  mark(3);
+  return s;
 }
 
 mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
@@ -685,6 +820,223 @@ mla_status mla_decode_profiled(const mla_config* cfg, const void* q, int32_t bat
   if (events == nullptr) return MLA_ERR_INVALID_ARG;
   return decode_impl(cfg, q, batch, tq, cache, num_pages, block_table, max_pages, seq_lens,
                      w_uk_t, w_uv, workspace, ws_bytes, out, stream, events);
+}
+
+size_t mla_query_workspace_size(const mla_config* cfg, int32_t q_lora, int32_t n_tok) {
+  if (check_config(cfg) != MLA_OK || q_lora < 1 || n_tok < 1) return 0;
+  return query_layout(cfg, q_lora, n_tok, nullptr).bytes;
+}
+
+mla_status mla_query(const mla_config* cfg, int32_t q_lora, const void* x, int32_t n_tok,
+                     const void* w_qa, const void* q_gain, const void* w_qb, void* workspace,
+                     size_t ws_bytes, void* q_out, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (q_lora < 1 || n_tok < 1 || n_tok > 65535) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, w_qa, q_gain, w_qb, workspace, q_out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(q_lora) * elem_bytes(cfg) % 16 != 0 ||
+      static_cast<int64_t>(cfg->d_model) * elem_bytes(cfg) % 16 != 0)
+    return MLA_ERR_UNSUPPORTED;
+  if (ws_bytes < mla_query_workspace_size(cfg, q_lora, n_tok)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const QueryLayout L = query_layout(cfg, q_lora, n_tok, workspace);
+  const int M_b = cfg->n_heads * (cfg->d_nope + cfg->d_rope);
+  const size_t rms_smem = static_cast<size_t>(q_lora) * sizeof(float);
+  if (rms_smem > 200 * 1024) return MLA_ERR_UNSUPPORTED;
+  if (tc_query_shape(cfg, q_lora)) {
+    // (1) q_a partial sums = x · w_qaᵀ, split over K; (2) sum + q_norm -> bf16 q_a;
+    // (3) q = q_a · w_qbᵀ -> bf16
+    const QueryPlan p = query_plan(cfg, q_lora, n_tok);
+    mla_status s = weight_gemm(w_qa, q_lora, cfg->d_model, x, n_tok, p.a, 1, p.bn,
+                               EpiSplitK{L.partial, n_tok, q_lora}, st);
+    if (s != MLA_OK) return s;
+    if (!allow_smem(rms_rows_kernel<__nv_bfloat16>, static_cast<int>(rms_smem))) return MLA_ERR_CUDA;
+    s = launch_pdl(rms_rows_kernel<__nv_bfloat16>, dim3(n_tok), dim3(256), rms_smem, st,
+                   static_cast<const float*>(L.partial), p.a.k_splits, static_cast<int>(n_tok),
+                   static_cast<int>(q_lora), static_cast<const __nv_bfloat16*>(q_gain),
+                   cfg->rms_eps, static_cast<__nv_bfloat16*>(L.qa));
+    if (s != MLA_OK) return s;
+    const SplitPlan sb = split_plan(1, 1, q_lora / 64, 1, false);   // whole K per CTA
+    return weight_gemm(w_qb, M_b, q_lora, L.qa, n_tok, sb, p.m_per_cta_b, p.bn,
+                       EpiStoreBf16{static_cast<__nv_bfloat16*>(q_out), M_b}, st);
+  }
+  // CUDA cores: fp32 sums, the same roundings
+  auto run = [&](auto tag) -> mla_status {
+    using T = decltype(tag);
+    linear_rows_kernel<T><<<dim3((q_lora + 7) / 8, n_tok), 256, 0, st>>>(
+        static_cast<const T*>(x), static_cast<const T*>(w_qa), L.partial, n_tok, q_lora,
+        cfg->d_model);
+    if (!allow_smem(rms_rows_kernel<T>, static_cast<int>(rms_smem))) return MLA_ERR_CUDA;
+    rms_rows_kernel<T><<<n_tok, 256, rms_smem, st>>>(L.partial, 1, n_tok, q_lora,
+                                                      static_cast<const T*>(q_gain),
+                                                      cfg->rms_eps, static_cast<T*>(L.qa));
+    linear_rows_kernel<T><<<dim3((M_b + 7) / 8, n_tok), 256, 0, st>>>(
+        static_cast<const T*>(L.qa), static_cast<const T*>(w_qb), L.q32, n_tok, M_b, q_lora);
+    const int64_t count = static_cast<int64_t>(n_tok) * M_b;
+    round_rows_kernel<T><<<static_cast<int>((count + 255) / 256 < 4096 ? (count + 255) / 256 : 4096),
+                           256, 0, st>>>(L.q32, count, static_cast<T*>(q_out));
+    return last_launch_status();
+  };
+  return cfg->dtype == MLA_DTYPE_F32 ? run(float{}) : run(__nv_bfloat16{});
+}
+
+size_t mla_output_workspace_size(const mla_config* cfg, int32_t n_tok) {
+  if (check_config(cfg) != MLA_OK || n_tok < 1) return 0;
+  return output_ws_bytes(cfg, n_tok);
+}
+
+mla_status mla_output(const mla_config* cfg, const void* attn, int32_t n_tok, const void* w_o,
+                      void* workspace, size_t ws_bytes, void* y, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (n_tok < 1 || n_tok > 65535) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {attn, w_o, workspace, y};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  const int K = cfg->n_heads * cfg->d_v;
+  if (static_cast<int64_t>(K) * elem_bytes(cfg) % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  if (ws_bytes < mla_output_workspace_size(cfg, n_tok)) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  float* partial = static_cast<float*>(workspace);
+  const int64_t count = static_cast<int64_t>(n_tok) * cfg->d_model;
+  const int sum_blocks = static_cast<int>((count + 255) / 256 < 4096 ? (count + 255) / 256 : 4096);
+  if (tc_output_shape(cfg)) {
+    const OutputPlan p = output_plan(cfg, n_tok);
+    const mla_status s = weight_gemm(w_o, cfg->d_model, K, attn, n_tok, p.s, 1, p.bn,
+                                     EpiSplitK{partial, n_tok, cfg->d_model}, st);
+    if (s != MLA_OK) return s;
+    return launch_pdl(sum_splits_kernel<__nv_bfloat16>, dim3(sum_blocks), dim3(256), 0, st,
+                      static_cast<const float*>(partial), p.s.k_splits, count,
+                      static_cast<__nv_bfloat16*>(y));
+  }
+  auto run = [&](auto tag) -> mla_status {
+    using T = decltype(tag);
+    linear_rows_kernel<T><<<dim3((cfg->d_model + 7) / 8, n_tok), 256, 0, st>>>(
+        static_cast<const T*>(attn), static_cast<const T*>(w_o), partial, n_tok, cfg->d_model, K);
+    sum_splits_kernel<T><<<sum_blocks, 256, 0, st>>>(partial, 1, count, static_cast<T*>(y));
+    return last_launch_status();
+  };
+  return cfg->dtype == MLA_DTYPE_F32 ? run(float{}) : run(__nv_bfloat16{});
+}
+
+mla_status mla_decode_partial(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                              const void* cache, int32_t num_pages, const int32_t* block_table,
+                              int32_t max_pages, const int32_t* seq_lens,
+                              const int32_t* kv_begin, const int32_t* kv_end, const void* w_uk_t,
+                              void* workspace, size_t ws_bytes, void* o_part, float* lse,
+                              void* stream) {
+  if (kv_begin == nullptr || kv_end == nullptr || o_part == nullptr || lse == nullptr)
+    return MLA_ERR_INVALID_ARG;
+  if (!aligned16(kv_begin) || !aligned16(kv_end)) return MLA_ERR_INVALID_ARG;
+  return decode_impl(cfg, q, batch, tq, cache, num_pages, block_table, max_pages, seq_lens,
+                     w_uk_t, nullptr, workspace, ws_bytes, nullptr, stream, nullptr, kv_begin,
+                     kv_end, o_part, lse);
+}
+
+size_t mla_combine_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq) {
+  if (check_config(cfg) != MLA_OK || batch < 1 || tq < 1) return 0;
+  if (tc_decode_shape(cfg)) return 0;
+  return align_up(static_cast<size_t>(batch) * tq * cfg->n_heads * cfg->d_c * sizeof(float));
+}
+
+mla_status mla_combine(const mla_config* cfg, int32_t n_parts, int32_t batch, int32_t tq,
+                       const void* o_parts, const float* lse_parts, const void* w_uv,
+                       void* workspace, size_t ws_bytes, void* out, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (n_parts < 1 || batch < 1 || tq < 1) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {o_parts, lse_parts, w_uv, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_combine_workspace_size(cfg, batch, tq);
+  if (ws_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  if (need > 0 && (workspace == nullptr || !aligned16(workspace))) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n_q = batch * tq;
+  const int rows = n_q * cfg->n_heads;
+  if (tc_decode_shape(cfg)) {
+    // the fused merge + value projection, reading the gathered parts in part order
+    VprojParams vp{static_cast<const __nv_bfloat16*>(o_parts), lse_parts, nullptr,
+                   static_cast<__nv_bfloat16*>(out), cfg->n_heads, tq, 1, n_q, cfg->d_v, n_parts};
+    return launch_vproj(cfg, w_uv, vp, st, false);
+  }
+  auto run = [&](auto tag) -> mla_status {
+    using T = decltype(tag);
+    float* o_lat = static_cast<float*>(workspace);
+    combine_simt_kernel<T><<<rows, 256, 0, st>>>(static_cast<const T*>(o_parts), lse_parts,
+                                                 n_parts, rows, cfg->d_c, o_lat);
+    outproj_simt_kernel<T><<<rows, 256, cfg->d_c * sizeof(float), st>>>(
+        o_lat, static_cast<const T*>(w_uv), static_cast<T*>(out), cfg->n_heads, cfg->d_c,
+        cfg->d_v);
+    return last_launch_status();
+  };
+  return cfg->dtype == MLA_DTYPE_F32 ? run(float{}) : run(__nv_bfloat16{});
+}
+
+// The tensor-core prefill: positions, the tcgen05 append, then decode with tq = t_new.
+static bool tc_prefill_shape(const mla_config* c) {
+  return tc_decode_shape(c) && tc_append_shape(c);
+}
+
+struct PrefillLayout {
+  int32_t *seq_idx, *pos;
+  void *app_ws, *dec_ws;
+  size_t app_bytes, dec_bytes, bytes;
+};
+static PrefillLayout prefill_layout(const mla_config* c, int batch, int t_new, void* ws) {
+  PrefillLayout L{};
+  Carve cv(ws);
+  const size_t n = static_cast<size_t>(batch) * t_new;
+  L.seq_idx = cv.take<int32_t>(n);
+  L.pos = cv.take<int32_t>(n);
+  L.app_bytes = mla_append_workspace_size(c, static_cast<int32_t>(n));
+  L.app_ws = cv.take<uint8_t>(L.app_bytes);
+  L.dec_bytes = mla_decode_workspace_size(c, batch, t_new);
+  L.dec_ws = cv.take<uint8_t>(L.dec_bytes);
+  L.bytes = cv.off;
+  return L;
+}
+
+size_t mla_prefill_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new) {
+  if (check_config(cfg) != MLA_OK || batch < 1 || t_new < 1) return 0;
+  if (!tc_prefill_shape(cfg)) return mla_prefill_ref_workspace_size(cfg, batch, t_new);
+  const PrefillLayout L = prefill_layout(cfg, batch, t_new, nullptr);
+  return (L.app_bytes == 0 || L.dec_bytes == 0) ? 0 : L.bytes;
+}
+
+mla_status mla_prefill(const mla_config* cfg, const void* x, const void* q, int32_t batch,
+                       int32_t t_new, const void* w_dkv, const void* kv_gain, const void* w_uk_t,
+                       const void* w_uv, const int32_t* seq_lens, const int32_t* block_table,
+                       int32_t max_pages, void* cache, int32_t num_pages, void* workspace,
+                       size_t ws_bytes, void* out, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (!tc_prefill_shape(cfg))
+    return mla_prefill_ref(cfg, x, q, batch, t_new, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens,
+                           block_table, max_pages, cache, num_pages, workspace, ws_bytes, out,
+                           stream);
+  if (batch < 1 || t_new < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(batch) * t_new > 65535) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens, block_table, cache,
+                        workspace, out};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  const size_t need = mla_prefill_workspace_size(cfg, batch, t_new);
+  if (need == 0) return MLA_ERR_INVALID_ARG;
+  if (ws_bytes < need) return MLA_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int n = batch * t_new;
+  const PrefillLayout L = prefill_layout(cfg, batch, t_new, workspace);
+  prefill_positions_kernel<<<(n + 255) / 256, 256, 0, st>>>(seq_lens, t_new, n, L.seq_idx, L.pos);
+  mla_status s = last_launch_status();
+  if (s != MLA_OK) return s;
+  s = mla_append_latent(cfg, x, n, w_dkv, kv_gain, L.seq_idx, L.pos, block_table, batch,
+                        max_pages, cache, num_pages, L.app_ws, L.app_bytes, stream);
+  if (s != MLA_OK) return s;
+  return decode_impl(cfg, q, batch, t_new, cache, num_pages, block_table, max_pages, seq_lens,
+                     w_uk_t, w_uv, L.dec_ws, L.dec_bytes, out, stream, nullptr);
 }
 
 size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new) {

@@ -187,6 +187,57 @@ append_finish_cluster_kernel(const float* __restrict__ kv, int n_splits, int n_t
   }
 }
 
+// ------------------------------------------------------- q path and output projection
+// The q path's normalisation (the module's q_norm after wq_a): per token n,
+//   out[n][f] = v[f] / sqrt(mean(v^2) + eps) * gain[f],  v[f] = sum_s partial[s][n][f]
+// with the split-K partials added in split order. One block per token.
+template <typename T>
+__global__ void __launch_bounds__(256)
+rms_rows_kernel(const float* __restrict__ partial, int n_splits, int n_tok, int F,
+                const T* __restrict__ gain, float eps, T* __restrict__ out) {
+  __shared__ float red[32];
+  extern __shared__ float row_s[];   // [F]
+  pdl_wait();   // the partials of the GEMM just before are complete from here on
+  const int n = blockIdx.x;
+  const int64_t stride = static_cast<int64_t>(n_tok) * F;
+  float ss = 0.0f;
+  for (int f = threadIdx.x; f < F; f += blockDim.x) {
+    const float* src = partial + static_cast<int64_t>(n) * F + f;
+    float v = 0.0f;
+    for (int s = 0; s < n_splits; ++s) v += src[s * stride];
+    row_s[f] = v;
+    ss = fmaf(v, v, ss);
+  }
+  ss = block_sum(ss, red);   // also orders the row_s writes before the reads below
+  const float rstd = 1.0f / sqrtf(ss / static_cast<float>(F) + eps);
+  for (int f = threadIdx.x; f < F; f += blockDim.x)
+    out[static_cast<int64_t>(n) * F + f] = Elem<T>::from_f(row_s[f] * rstd * Elem<T>::to_f(gain[f]));
+}
+
+// out[i] = sum_s partial[s][i] in split order, rounded to T (the output projection's split-K
+// sum). Grid-stride over the n_tok * F outputs.
+template <typename T>
+__global__ void __launch_bounds__(256)
+sum_splits_kernel(const float* __restrict__ partial, int n_splits, int64_t count,
+                  T* __restrict__ out) {
+  pdl_wait();
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v = 0.0f;
+    for (int s = 0; s < n_splits; ++s) v += partial[s * count + i];
+    out[i] = Elem<T>::from_f(v);
+  }
+}
+
+// Rows of fp32 values rounded to T (the SIMT q path's up-projection output).
+template <typename T>
+__global__ void __launch_bounds__(256)
+round_rows_kernel(const float* __restrict__ in, int64_t count, T* __restrict__ out) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < count;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    out[i] = Elem<T>::from_f(in[i]);
+}
+
 // ---------------------------------------------------- decode on CUDA cores (fp32 arithmetic)
 // Query rows are r = (b*Tq + t)*H + h. The length of sequence b must lie in [Tq, max_pos].
 __device__ __forceinline__ bool length_ok(int L, int Tq, int max_pos) {
@@ -228,14 +279,16 @@ qabs_simt_kernel(const T* __restrict__ q, const T* __restrict__ w_uk_t,
 }
 
 // One block per query row: online softmax over chunks of 256 keys.
-//   s_j = scale * qhat · cache_row_j  (all d_c + d_r dims),  j <= L_b - Tq + t
+//   s_j = scale * qhat · cache_row_j  (all d_c + d_r dims),  j in the row's visible_keys range
 //   o_lat = sum_j softmax(s)_j * cache_row_j[:d_c]
+// lse_out (optional): natural-log log-sum-exp of the row's scores, -inf if it sees no key.
 template <typename T>
 __global__ void __launch_bounds__(256)
 attn_simt_kernel(const float* __restrict__ qhat, const T* __restrict__ cache,
                  const int32_t* __restrict__ block_table, const int32_t* __restrict__ seq_lens,
                  float* __restrict__ o_lat, int H, int Tq, int d_c, int d_r, int max_pages,
-                 int num_pages, int page_size, float scale) {
+                 int num_pages, int page_size, float scale, KeyRange keys,
+                 float* __restrict__ lse_out) {
   constexpr int CH = 256;
   __shared__ float red[32];
   __shared__ float p_s[CH];
@@ -250,18 +303,20 @@ attn_simt_kernel(const float* __restrict__ qhat, const T* __restrict__ cache,
   float* out = o_lat + static_cast<int64_t>(r) * d_c;
   if (!length_ok(L, Tq, max_pages * page_size)) {
     for (int c = threadIdx.x; c < d_c; c += blockDim.x) out[c] = 0.0f;
+    if (threadIdx.x == 0 && lse_out != nullptr) lse_out[r] = -INFINITY;
     if (threadIdx.x == 0 && (r % H) == 0 && t == 0) record_error(MLA_ERR_DEVICE_BAD_LENGTH);
     return;
   }
-  const int n_keys = L - Tq + t + 1;
+  int k_lo, k_hi;
+  visible_keys(keys, b, L, Tq, t, &k_lo, &k_hi);
   for (int i = threadIdx.x; i < row; i += blockDim.x) qs[i] = qhat[static_cast<int64_t>(r) * row + i];
   for (int c = threadIdx.x; c < d_c; c += blockDim.x) acc[c] = 0.0f;
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
   float m = -INFINITY, l = 0.0f;
   bool oob = false;
-  for (int j0 = 0; j0 < n_keys; j0 += CH) {
-    const int cnt = min(CH, n_keys - j0);
+  for (int j0 = k_lo; j0 <= k_hi; j0 += CH) {
+    const int cnt = min(CH, k_hi - j0 + 1);
     for (int jj = threadIdx.x; jj < cnt; jj += blockDim.x) {
       const int j = j0 + jj;
       const int page = block_table[static_cast<int64_t>(b) * max_pages + j / page_size];
@@ -307,6 +362,32 @@ attn_simt_kernel(const float* __restrict__ qhat, const T* __restrict__ cache,
   if (oob) record_error(MLA_ERR_DEVICE_OOB);
   const float inv = (l > 0.0f) ? 1.0f / l : 0.0f;
   for (int c = threadIdx.x; c < d_c; c += blockDim.x) out[c] = acc[c] * inv;
+  if (threadIdx.x == 0 && lse_out != nullptr) lse_out[r] = (l > 0.0f) ? m + logf(l) : -INFINITY;
+}
+
+// Merge of n_parts partial decodes over disjoint key ranges (rows r, natural-log lse):
+//   o_lat[r][:] = sum_k e^(lse_k - m) O_k[r][:] / sum_k e^(lse_k - m), in part order.
+// One block per row; zeros when no part saw a key.
+template <typename T>
+__global__ void __launch_bounds__(256)
+combine_simt_kernel(const T* __restrict__ o_parts, const float* __restrict__ lse_parts,
+                    int n_parts, int rows, int d_c, float* __restrict__ o_lat) {
+  const int r = blockIdx.x;
+  float m = -INFINITY;
+  for (int k = 0; k < n_parts; ++k) m = fmaxf(m, lse_parts[static_cast<int64_t>(k) * rows + r]);
+  float den = 0.0f;
+  if (m > -INFINITY)
+    for (int k = 0; k < n_parts; ++k) den += expf(lse_parts[static_cast<int64_t>(k) * rows + r] - m);
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  for (int c = threadIdx.x; c < d_c; c += blockDim.x) {
+    float a = 0.0f;
+    if (m > -INFINITY)
+      for (int k = 0; k < n_parts; ++k) {
+        const int64_t i = static_cast<int64_t>(k) * rows + r;
+        a = fmaf(expf(lse_parts[i] - m), Elem<T>::to_f(o_parts[i * d_c + c]), a);
+      }
+    o_lat[static_cast<int64_t>(r) * d_c + c] = a * inv;
+  }
 }
 
 // out[r][v] = sum_c o_lat[r][c] * w_uv[h][v][c]. One warp per output column v.

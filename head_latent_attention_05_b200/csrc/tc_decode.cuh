@@ -64,7 +64,7 @@ constexpr float ATT_RESCALE_THRESHOLD = 8.0f;     // log2 units
 
 struct AttnSeg {
   int32_t unit;        // b * n_mt + mt
-  int32_t tile_begin;  // first 64-token page of the segment
+  int32_t tile_begin;  // first 64-token page of the segment (page index within the sequence)
   int32_t tile_end;    // one past the last
   int32_t pair;        // CTA pair that runs it
 };
@@ -80,13 +80,16 @@ struct AttnParams {
   int max_pages, num_pages;
   int H, Tq, R, n_mt;
   float scale_log2;          // softmax_scale * log2(e)
+  KeyRange keys;             // keys each query row may see (causal, window, key range)
 };
 
 // ------------------------------------------------------------------------ split-KV planner
 
 struct PlanParams {
   const int32_t* seq_lens;
-  int B, Tq, n_mt, max_pos, P, max_segs;
+  int B, Tq, H, n_mt, max_pos, P, max_segs;
+  KeyRange keys;
+  int32_t* unit_first;   // [U] scratch: first page of each unit's key range
   int32_t* unit_tiles;   // [U] scratch: first global tile of each unit
   int32_t* unit_seg;     // [U + 1]
   int32_t* pair_seg;     // [P + 1]
@@ -143,6 +146,11 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
 // The planner, run by one whole block of any size (a multiple of 32): it rides along as an
 // extra block of the query-absorption GEMM, which runs just before the attention kernel.
 //
+// Pages of a unit. A unit's rows are query tokens t0..t1 of one sequence (all heads of each);
+// the unit covers the pages from the one holding the first key its first token sees to the one
+// holding the last key its last token sees (visible_keys: causal, window, key range), so a
+// prefill's early tokens and a windowed decode skip the pages none of their rows can see.
+//
 // Balance. A CTA pair pays a fixed price each time it moves on to another unit (the finished
 // segment's epilogue and the next unit's Q̂ load lie on its critical path; measured at about
 // five tiles' worth on B200). So the tile list is cut in a virtual stream in which every unit
@@ -165,13 +173,23 @@ __device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
     const int u = u0 + threadIdx.x;
     int n = 0;
     if (u < U) {
-      const int b = u / pp.n_mt;
+      const int b = u / pp.n_mt, mt = u % pp.n_mt;
       const int L = pp.seq_lens[b];
+      int first = 0;
       if (L >= pp.Tq && L <= pp.max_pos) {
-        n = (L + ATT_PAGE - 1) / ATT_PAGE;
-      } else if (u % pp.n_mt == 0) {
+        const int t0 = (mt * 128) / pp.H;
+        const int t1 = min(pp.Tq - 1, (mt * 128 + 127) / pp.H);
+        int lo0, hi0, lo1, hi1;
+        visible_keys(pp.keys, b, L, pp.Tq, t0, &lo0, &hi0);
+        visible_keys(pp.keys, b, L, pp.Tq, t1, &lo1, &hi1);
+        if (hi1 >= lo0) {
+          first = lo0 / ATT_PAGE;
+          n = hi1 / ATT_PAGE + 1 - first;
+        }
+      } else if (mt == 0) {
         record_error(MLA_ERR_DEVICE_BAD_LENGTH);
       }
+      pp.unit_first[u] = first;
     }
     int excl;
     const int tot = block_exclusive_scan(n, &excl, warp_tot);
@@ -213,8 +231,8 @@ __device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
         if (e <= a) continue;
         AttnSeg sg;
         sg.unit = u;
-        sg.tile_begin = a - v0;
-        sg.tile_end = e - v0;
+        sg.tile_begin = pp.unit_first[u] + (a - v0);
+        sg.tile_end = pp.unit_first[u] + (e - v0);
         sg.pair = p;
         if (s0 + i < pp.max_segs) pp.segs[s0 + i] = sg;
         atomicMin(&first_seg[p], s0 + i);
@@ -595,7 +613,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         const int L = p.seq_lens[b];
         const int r_in = mt * 128 + r_local;
         const bool row_valid = r_in < p.R;
-        const int limit = L - p.Tq + (row_valid ? r_in / p.H : 0);   // last key this row sees
+        // keys this row sees (lo > hi: none), and the union over the unit's rows
+        int lo_row = 1, hi_row = 0, lo_u, hi_u, unused;
+        if (row_valid) visible_keys(p.keys, b, L, p.Tq, r_in / p.H, &lo_row, &hi_row);
+        visible_keys(p.keys, b, L, p.Tq, (mt * 128) / p.H, &lo_u, &unused);
+        visible_keys(p.keys, b, L, p.Tq, min(p.Tq - 1, (mt * 128 + 127) / p.H), &unused, &hi_u);
         float m_ref = -INFINITY, l_part = 0.0f;
         for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
           if (!att_warp_wait(sh, &sh.s_full, g & 1)) { ok = false; break; }
@@ -606,12 +628,12 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.s_free);
-          // this thread's visible columns: 0 .. nvis-1 of its 32
+          // this thread's visible columns: c_lo .. c_hi of its 32 (none if c_lo > c_hi)
           const int j0 = tile * ATT_PAGE + hc * 32;
-          const int jmax = row_valid ? min(limit, L - 1) : -1;   // inclusive
-          const int nvis = max(0, min(32, jmax - j0 + 1));
+          const int c_lo = max(0, lo_row - j0), c_hi = min(31, hi_row - j0);
+          const bool all_vis = c_lo == 0 && c_hi == 31;
           float mx0 = -INFINITY, mx1 = -INFINITY;
-          if (nvis == 32) {
+          if (all_vis) {
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
               mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
@@ -620,8 +642,9 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           } else {
 #pragma unroll
             for (int c = 0; c < 32; c += 2) {
-              mx0 = fmaxf(mx0, c < nvis ? __uint_as_float(sr[c]) : -INFINITY);
-              mx1 = fmaxf(mx1, c + 1 < nvis ? __uint_as_float(sr[c + 1]) : -INFINITY);
+              mx0 = fmaxf(mx0, (c >= c_lo && c <= c_hi) ? __uint_as_float(sr[c]) : -INFINITY);
+              mx1 = fmaxf(mx1, (c + 1 >= c_lo && c + 1 <= c_hi) ? __uint_as_float(sr[c + 1])
+                                                                 : -INFINITY);
             }
           }
           // agree on the row maximum with the partner warp (same rows, other 32 columns)
@@ -670,9 +693,9 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
               const int c = q * 8 + 2 * e;
               float x0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
               float x1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
-              if (nvis < 32) {
-                x0 = c < nvis ? x0 : 0.0f;
-                x1 = c + 1 < nvis ? x1 : 0.0f;
+              if (!all_vis) {
+                x0 = (c >= c_lo && c <= c_hi) ? x0 : 0.0f;
+                x1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? x1 : 0.0f;
               }
               ps0 += x0;
               ps1 += x1;
@@ -683,16 +706,19 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                 make_uint4(w[0], w[1], w[2], w[3]);
           }
           l_part += ps0 + ps1;
-          // rows past the sequence end must be zero in the value chunks (P is 0 there, but
-          // stale cache contents could be non-finite); S is done, so they have landed
-          const int valid_tok = L - tile * ATT_PAGE;
-          if (valid_tok < ATT_PAGE) {
+          // rows outside the keys any row of the unit sees must be zero in the value chunks
+          // (P is 0 there, but stale slots past the sequence end, or slots outside a key range,
+          // could hold non-finite values); S is done, so they have landed. Kept: [z_lo, z_keep).
+          const int z_lo = min(ATT_PAGE, max(0, lo_u - tile * ATT_PAGE));
+          const int z_keep = max(z_lo, min(ATT_PAGE, hi_u + 1 - tile * ATT_PAGE));
+          const int nz = z_lo + (ATT_PAGE - z_keep);
+          if (nz > 0) {
             uint8_t* vbase = stage_buf + (g % ATT_STAGES) * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES;
-            const int nrows = ATT_PAGE - valid_tok;
-            for (int i = t_idx; i < 4 * nrows * 8; i += 256) {
-              const int chunk = i / (nrows * 8);
-              const int rem = i % (nrows * 8);
-              const int row = valid_tok + rem / 8, piece = rem % 8;
+            for (int i = t_idx; i < 4 * nz * 8; i += 256) {
+              const int chunk = i / (nz * 8);
+              const int rem = i % (nz * 8);
+              const int ri = rem / 8, piece = rem % 8;
+              const int row = ri < z_lo ? ri : z_keep + (ri - z_lo);
               *reinterpret_cast<uint4*>(vbase + chunk * ATT_CHUNK_BYTES + row * 128 + piece * 16) =
                   make_uint4(0, 0, 0, 0);
             }

@@ -213,6 +213,22 @@ struct EpiSplitK {
   }
 };
 
+// Plain store: out[n][m] = v rounded to bf16, rows of `ld` elements (the q path's up-projection
+// wq_b, whose M side is the n_heads * (d_nope + d_rope) query features of each token).
+struct EpiStoreBf16 {
+  __nv_bfloat16* out;
+  int ld;
+  struct SideState {};
+  __host__ __device__ static constexpr int side_bytes(int) { return 0; }
+  __device__ void aux() const {}
+  __device__ SideState side_begin(int, int, int) const { return {}; }
+  __device__ void side_issue(const CUtensorMap*, uint8_t*, uint64_t*, int, int) const {}
+  __device__ void side(int, int, int, int, int, const SideState&, const uint8_t*, uint64_t*) const {}
+  __device__ void operator()(int, int, int m, int n, float v) const {
+    out[static_cast<int64_t>(n) * ld + m] = __float2bfloat16_rn(v);
+  }
+};
+
 // Absorbed query: qhat[(n*H + h)][m] = q_lat (bf16), m < d_c. Warps 2-3 of the n-tile-0 CTA of
 // head h also write the rotated rope part qhat[..][d_c + i] while the MMAs run, and the one aux
 // block runs the split-KV planner of the attention kernel that follows.

@@ -15,12 +15,18 @@
 
 namespace mla {
 
+// Two sources of partials. Segment mode (n_parts == 0): the attention kernel's per-segment O / l
+// [segments][128][512] with base-2 lse [segments][128], a row's segments listed by unit_seg.
+// Parts mode (n_parts > 0): n_parts full sets of rows [n_parts][n_q * H][512] with natural-log
+// lse [n_parts][n_q * H] (the partial decodes of several GPUs over disjoint key ranges,
+// gathered), merged in part order.
 struct VprojParams {
-  const __nv_bfloat16* o_part;  // [segments][128][512] per-segment O / l (bf16)
-  const float* lse;           // [segments][128] base-2 log-sum-exp of each partial
-  const int32_t* unit_seg;    // [U + 1] first segment of each unit
-  __nv_bfloat16* out;         // [n_q][H][d_v]
+  const __nv_bfloat16* o_part;  // partial O / l (bf16), see above
+  const float* lse;             // their log-sum-exp, see above
+  const int32_t* unit_seg;      // [U + 1] first segment of each unit (segment mode)
+  __nv_bfloat16* out;           // [n_q][H][d_v]
   int H, Tq, n_mt, n_q, d_v;
+  int n_parts;                  // 0: segment mode
 };
 
 constexpr int VP_THREADS = 256;
@@ -76,19 +82,30 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
   // K-chunk 2i + k/8.
   constexpr int RP = 16, TPR = VP_THREADS / RP, PASSES = BN / RP;
   const int rr_l = threadIdx.x / TPR, k = threadIdx.x % TPR;
-  // the segment lists were written two kernels back (by the planner): read them before waiting
-  int seg0[PASSES], seg1[PASSES], rowl[PASSES];
+  // each row's partials: cnt of them, the first at row base of the partial arrays, then every
+  // `stride` rows. The segment lists were written two kernels back (by the planner): read them
+  // before waiting.
+  const int64_t stride = p.n_parts > 0 ? static_cast<int64_t>(p.n_q) * p.H : 128;
+  const float lse_scale = p.n_parts > 0 ? 1.4426950408889634f : 1.0f;   // to base 2
+  int64_t base[PASSES];
+  int cnt[PASSES];
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int n = n0 + ps * RP + rr_l;
-    seg0[ps] = seg1[ps] = rowl[ps] = 0;
+    base[ps] = 0;
+    cnt[ps] = 0;
     if (n < p.n_q) {
-      const int b = n / p.Tq, t = n % p.Tq;
-      const int r = t * p.H + h;
-      const int u = b * p.n_mt + r / 128;
-      seg0[ps] = p.unit_seg[u];
-      seg1[ps] = p.unit_seg[u + 1];
-      rowl[ps] = r % 128;
+      if (p.n_parts > 0) {
+        base[ps] = static_cast<int64_t>(n) * p.H + h;
+        cnt[ps] = p.n_parts;
+      } else {
+        const int b = n / p.Tq, t = n % p.Tq;
+        const int r = t * p.H + h;
+        const int u = b * p.n_mt + r / 128;
+        const int s0 = p.unit_seg[u];
+        base[ps] = static_cast<int64_t>(s0) * 128 + r % 128;
+        cnt[ps] = p.unit_seg[u + 1] - s0;
+      }
     }
   }
   pdl_wait();   // the attention partials are complete and visible from here on
@@ -96,9 +113,11 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int rr = ps * RP + rr_l;
-    const int s0 = seg0[ps], s1 = seg1[ps], rl = rowl[ps];
+    const int s1 = cnt[ps];
+    const int64_t rb = base[ps];
+    auto lse_of = [&](int s) { return p.lse[rb + s * stride] * lse_scale; };
     float mx = -INFINITY;
-    for (int s = s0 + k; s < s1; s += TPR) mx = fmaxf(mx, p.lse[static_cast<int64_t>(s) * 128 + rl]);
+    for (int s = k; s < s1; s += TPR) mx = fmaxf(mx, lse_of(s));
 #pragma unroll
     for (int o = TPR / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     float den = 0.0f;
@@ -106,9 +125,9 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
 #pragma unroll
     for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
     if (mx > -INFINITY) {
-      for (int s = s0 + k; s < s1; s += TPR) den += exp2f(p.lse[static_cast<int64_t>(s) * 128 + rl] - mx);
-      // four segments' loads in flight at a time; the sum runs in segment order
-      for (int sb = s0; sb < s1; sb += 4) {
+      for (int s = k; s < s1; s += TPR) den += exp2f(lse_of(s) - mx);
+      // four partials' loads in flight at a time; the sum runs in partial order
+      for (int sb = 0; sb < s1; sb += 4) {
         float w[4];
         uint4 v[4][4];
 #pragma unroll
@@ -116,9 +135,8 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
           const int s = sb + j;
           w[j] = 0.0f;
           if (s < s1) {
-            w[j] = exp2f(p.lse[static_cast<int64_t>(s) * 128 + rl] - mx);
-            const uint4* src = reinterpret_cast<const uint4*>(
-                p.o_part + (static_cast<int64_t>(s) * 128 + rl) * ATT_DC);
+            w[j] = exp2f(lse_of(s) - mx);
+            const uint4* src = reinterpret_cast<const uint4*>(p.o_part + (rb + s * stride) * ATT_DC);
 #pragma unroll
             for (int i = 0; i < 4; ++i) v[j][i] = src[k + TPR * i];
           }
@@ -213,6 +231,49 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
     tc_fence_after_sync();
     tmem_dealloc(tmem, TMEM_COLS);
   }
+}
+
+// Merge of the attention kernel's per-segment partials into one partial per query row, for a
+// decode over a key range whose result another GPU's partials will be combined with:
+//   o_out[row][:] = sum_s 2^(lse_s - m) O_s / sum_s 2^(lse_s - m),   lse_out[row] = (m +
+//   log2(sum_s 2^(lse_s - m))) * ln 2  (natural log), -inf and zeros when the row saw no key.
+// Rows are row = n * H + h (n = b * Tq + t); 64 threads per row, 8 dims each, 4 rows a block.
+__global__ void __launch_bounds__(256)
+merge_partials_kernel(const __nv_bfloat16* __restrict__ o_seg, const float* __restrict__ lse_seg,
+                      const int32_t* __restrict__ unit_seg, int rows, int R, int n_mt,
+                      __nv_bfloat16* __restrict__ o_out, float* __restrict__ lse_out) {
+  pdl_wait();
+  const int row = blockIdx.x * 4 + static_cast<int>(threadIdx.x >> 6);
+  const int k = threadIdx.x & 63;
+  if (row >= rows) return;
+  const int b = row / R, r_in = row % R;
+  const int u = b * n_mt + r_in / 128, rl = r_in % 128;
+  const int s0 = unit_seg[u], s1 = unit_seg[u + 1];
+  float mx = -INFINITY;
+  for (int s = s0; s < s1; ++s) mx = fmaxf(mx, lse_seg[static_cast<int64_t>(s) * 128 + rl]);
+  float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  float den = 0.0f;
+  if (mx > -INFINITY) {
+    for (int s = s0; s < s1; ++s) {
+      const float w = exp2f(lse_seg[static_cast<int64_t>(s) * 128 + rl] - mx);
+      den += w;
+      const uint4 v = reinterpret_cast<const uint4*>(
+          o_seg + (static_cast<int64_t>(s) * 128 + rl) * ATT_DC)[k];
+      const uint32_t q[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&q[e]));
+        acc[2 * e] = fmaf(w, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(w, f.y, acc[2 * e + 1]);
+      }
+    }
+  }
+  const float inv = den > 0.0f ? 1.0f / den : 0.0f;
+  reinterpret_cast<uint4*>(o_out + static_cast<int64_t>(row) * ATT_DC)[k] = make_uint4(
+      pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+      pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+  if (k == 0)
+    lse_out[row] = den > 0.0f ? (mx + log2f(den)) * 0.6931471805599453f : -INFINITY;
 }
 
 }  // namespace mla

@@ -65,7 +65,13 @@ typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1 } mla_dtype;
  * rope_theta is the RoPE base: pair i of a d_rope-wide vector at position p turns by
  * p * rope_theta^(-2i/d_rope) (「淺析DeepSeek多頭潛在注意力機制（MLA）」, "MLA與ROPE的融合";
  * pairs are adjacent elements (2i, 2i+1)). page_size is the number of tokens per cache page.
- * Every entry point rejects d_rope > 128 with MLA_ERR_UNSUPPORTED.
+ * window limits attention to the most recent keys: with window > 0 a query at position p sees
+ * the keys p - window + 1 .. p only (the sliding-window "Streaming-MLA" variant, which keeps the
+ * last 1024 latents, in 「Multi-Head Latent Attention（MLA）原理与工程实践全解析」 §7); 0 means
+ * every earlier key (plain causal attention). The window applies to every decode and prefill
+ * entry point; appends are unaffected.
+ * Every entry point rejects d_rope > 128 with MLA_ERR_UNSUPPORTED, window < 0 with
+ * MLA_ERR_INVALID_ARG.
  */
 typedef struct {
   int32_t n_heads;
@@ -79,6 +85,7 @@ typedef struct {
   float softmax_scale;
   float rms_eps;
   float rope_theta;
+  int32_t window; /* 0 = unlimited */
 } mla_config;
 
 /* Human-readable name of a status code (static string). */
@@ -172,6 +179,111 @@ mla_status mla_decode_profiled(const mla_config* cfg, const void* q, int32_t bat
                                int32_t max_pages, const int32_t* seq_lens, const void* w_uk_t,
                                const void* w_uv, void* workspace, size_t ws_bytes, void* out,
                                void* stream, void* const* events);
+
+/* Bytes of workspace mla_query needs for n_tok tokens (0 if the arguments are invalid). */
+size_t mla_query_workspace_size(const mla_config* cfg, int32_t q_lora, int32_t n_tok);
+
+/*
+ * The query path of the module (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2: wq_a, q_norm,
+ * wq_b), producing the un-rotated per-head queries that mla_decode takes:
+ *     q_a = x · w_qaᵀ                                              (q_lora outputs, fp32 sums)
+ *     q_a = q_a / sqrt(mean(q_a^2) + rms_eps) * q_gain, rounded once to cfg->dtype
+ *     q   = q_a · w_qbᵀ, viewed as [n_heads][d_nope + d_rope], rounded to cfg->dtype
+ *   x       [n_tok, d_model]
+ *   w_qa    [q_lora, d_model]                      (wq_a weight)
+ *   q_gain  [q_lora]                               (q_norm weight)
+ *   w_qb    [n_heads * (d_nope + d_rope), q_lora]  (wq_b weight; per head [q_nope | q_rope])
+ *   workspace >= mla_query_workspace_size(cfg, q_lora, n_tok) bytes, 256-byte aligned
+ *   q_out   [n_tok, n_heads, d_nope + d_rope]
+ * bf16 with d_model and q_lora multiples of 64 runs two tcgen05 weight-streaming GEMMs (the
+ * first split over K) around a normalisation kernel; other shapes and fp32 run on CUDA cores.
+ * The pre-absorbed form (W_UK folded into wq_b) is not offered: at DeepSeek-V2 shape its weight
+ * is five times the bytes of wq_b's no-rope part plus W_UK, and decode streams every byte.
+ */
+mla_status mla_query(const mla_config* cfg, int32_t q_lora, const void* x, int32_t n_tok,
+                     const void* w_qa, const void* q_gain, const void* w_qb, void* workspace,
+                     size_t ws_bytes, void* q_out, void* stream);
+
+/* Bytes of workspace mla_output needs for n_tok tokens (0 if the arguments are invalid). */
+size_t mla_output_workspace_size(const mla_config* cfg, int32_t n_tok);
+
+/*
+ * The module's output projection wo (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2): the
+ * heads' outputs laid side by side, head after head, times woᵀ:
+ *     y[n][m] = sum_{h, v} w_o[m][h * d_v + v] * attn[n][h][v]     (fp32 sums, one rounding)
+ *   attn    [n_tok, n_heads, d_v]          (mla_decode's out)
+ *   w_o     [d_model, n_heads * d_v]       (wo weight)
+ *   workspace >= mla_output_workspace_size(cfg, n_tok) bytes, 256-byte aligned
+ *   y       [n_tok, d_model]
+ * bf16 with n_heads * d_v a multiple of 64 runs a split-K tcgen05 GEMM whose partial sums are
+ * added in split order; other shapes and fp32 run on CUDA cores. The variant with W_UV folded
+ * into wo is not offered: its weight (d_model x n_heads*d_c) is four times wo's at V2 shape.
+ */
+mla_status mla_output(const mla_config* cfg, const void* attn, int32_t n_tok, const void* w_o,
+                      void* workspace, size_t ws_bytes, void* y, void* stream);
+
+/*
+ * Decode over a share of each sequence's keys, for a long context whose cache is split over
+ * several GPUs (each holds whole pages of a key range): the same attention as mla_decode, but
+ * only keys kv_begin[b] <= j < kv_end[b] are read (with the causal rule and cfg->window), and
+ * the result is the partial latent output and its log-sum-exp instead of the projected output:
+ *     o_part[row][:] = sum_j softmax_j o_j  over the visible keys of the range (O / l),
+ *     lse[row]       = ln sum_j exp(s_j)    (natural log of the scaled scores; -inf and a zero
+ *                                            row when the range holds no key the row sees)
+ * with row = (b * tq + t) * n_heads + h. Partials of disjoint ranges that cover every key are
+ * merged by mla_combine into exactly mla_decode's result (up to rounding): the split-KV merge of
+ * this library, moved across GPUs. Pages outside [kv_begin, kv_end) are never read, so their
+ * block-table entries may be anything. The ranges should start on page boundaries (a page whose
+ * keys straddle two ranges is read by both GPUs).
+ *   kv_begin, kv_end  [batch] int32 (device), 0 <= kv_begin[b], kv_end[b] <= seq_lens[b]
+ *   o_part  [batch * tq * n_heads, d_c] in cfg->dtype;  lse [batch * tq * n_heads] float
+ *   other arguments and the workspace as in mla_decode (mla_decode_workspace_size)
+ * w_uv is not needed. Shapes and dtypes as mla_decode.
+ */
+mla_status mla_decode_partial(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
+                              const void* cache, int32_t num_pages, const int32_t* block_table,
+                              int32_t max_pages, const int32_t* seq_lens,
+                              const int32_t* kv_begin, const int32_t* kv_end, const void* w_uk_t,
+                              void* workspace, size_t ws_bytes, void* o_part, float* lse,
+                              void* stream);
+
+/* Bytes of workspace mla_combine needs (0 if the arguments are invalid). */
+size_t mla_combine_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq);
+
+/*
+ * Merge n_parts partial results of mla_decode_partial (one per key range, typically gathered
+ * from the GPUs that hold the ranges) and project:
+ *     o_lat[row] = sum_k e^(lse_k - m) o_part_k[row] / sum_k e^(lse_k - m),  m = max_k lse_k
+ *     out[b][t][h][:] = o_lat[row] · W_UV[h]ᵀ
+ * The parts are added in index order, so every GPU that runs this on the same gathered parts
+ * gets the same bits. A row that no part saw any key of gets zeros.
+ *   o_parts [n_parts, batch * tq * n_heads, d_c] in cfg->dtype
+ *   lse_parts [n_parts, batch * tq * n_heads] float
+ *   w_uv [n_heads, d_v, d_c];  out [batch, tq, n_heads, d_v]
+ *   workspace >= mla_combine_workspace_size(cfg, batch, tq) bytes (may be 0)
+ */
+mla_status mla_combine(const mla_config* cfg, int32_t n_parts, int32_t batch, int32_t tq,
+                       const void* o_parts, const float* lse_parts, const void* w_uv,
+                       void* workspace, size_t ws_bytes, void* out, void* stream);
+
+/* Bytes of workspace mla_prefill needs (0 if the arguments are invalid). */
+size_t mla_prefill_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new);
+
+/*
+ * Prefill on the tensor cores: append t_new tokens per sequence (as mla_append_latent) and
+ * return the attention outputs of all of them, each new token seeing the keys up to its own
+ * position (the prompt pass of 「淺析DeepSeek多頭潛在注意力機制（MLA）」, "大模型的整體推理過程",
+ * done token-causal, in the absorbed form). Same arguments and results as mla_prefill_ref. For
+ * bf16 at DeepSeek-V2 latent shapes (those mla_decode runs on tcgen05) the append is the
+ * tcgen05 down-projection and the attention is mla_decode's latent attention kernel with
+ * tq = t_new, each 128-row unit of query rows reading only the pages its tokens can see; other
+ * shapes run mla_prefill_ref's CUDA-core path.
+ */
+mla_status mla_prefill(const mla_config* cfg, const void* x, const void* q, int32_t batch,
+                       int32_t t_new, const void* w_dkv, const void* kv_gain, const void* w_uk_t,
+                       const void* w_uv, const int32_t* seq_lens, const int32_t* block_table,
+                       int32_t max_pages, void* cache, int32_t num_pages, void* workspace,
+                       size_t ws_bytes, void* out, void* stream);
 
 /* Bytes of workspace mla_prefill_ref needs (0 if the arguments are invalid). */
 size_t mla_prefill_ref_workspace_size(const mla_config* cfg, int32_t batch, int32_t t_new);

@@ -52,7 +52,7 @@ class Case:
 
 
 def make_case(w: W.Workload, lens: torch.Tensor | None = None, tail_fill=None,
-              device="cuda") -> Case:
+              device="cuda", window: int = 0) -> Case:
     lens = W.seq_lens(w) if lens is None else lens.to(torch.int32)
     pt = W.page_table(w, lens)
     weights = W.weights(w)
@@ -62,6 +62,7 @@ def make_case(w: W.Workload, lens: torch.Tensor | None = None, tail_fill=None,
             cache[page, slot:] = tail_fill
     x_new, seq_idx, pos, q = W.new_token_inputs(w, lens)
     cfg = config_of(w)
+    cfg.window = window
     d = dict(
         cache=cache.to(device), block_table=pt.block_table.to(device),
         seq_lens=lens.to(device), x_new=x_new.to(device), seq_idx=seq_idx.to(device),
@@ -108,11 +109,12 @@ def oracle_rows_of(c: Case, b: int, new_rows: np.ndarray) -> np.ndarray:
 
 
 def oracle_out(c: Case, b: int, heads, new_rows: np.ndarray) -> np.ndarray:
-    """Oracle output [Tq, len(heads), d_v] for sequence b (expanded form)."""
+    """Oracle output [Tq, len(heads), d_v] for sequence b (expanded form, the case's window)."""
     w = c.w
     W_UK, W_UV = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
     rows = oracle_rows_of(c, b, new_rows)
-    return O.decode_expanded(c.q[b], rows, W_UK, W_UV, w.scale, w.rope_theta, heads=heads)
+    return O.decode_expanded(c.q[b], rows, W_UK, W_UV, w.scale, w.rope_theta, heads=heads,
+                             window=int(c.cfg.window))
 
 
 def plant_score_staircase(c: Case, b: int, h: int, t: int = 0, base: float = 8.0,
