@@ -268,8 +268,8 @@ def output_projection(out, w_o) -> np.ndarray:
     """The module's output projection wo applied to per-head attention outputs.
 
     「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」 §2: the heads' outputs are laid side by side,
-    head after head (transpose to (seq, heads, d_v), then view as heads * d_v), and wo, an
-    nn.Linear(heads * d_v, dim) without bias, maps them back to the model width.
+    head after head, into one vector of heads * d_v values per token, and wo, a bias-free linear
+    map from heads * d_v to the model width, brings them back to d_model.
     out [..., H, d_v], w_o [d_model, H * d_v]; returns [..., d_model].
     """
     out = f64(out)
