@@ -14,23 +14,31 @@
 // exchanging partial scores through distributed shared memory instead of recomputing them
 // measured slower on B200 (DSMEM moves ~8 bytes/clock per SM).
 //
-// Per CTA: TMEM columns [0,256) O half, [256,320) S, [320,512) Q̂[:, 0:384] as bf16 pairs (the
-// A operand of the first 24 K-steps of S). Shared memory: 2 stages x 9 chunks of
-// [64 tokens x 64 dims] (the whole 576-wide page, 128-byte swizzle, one TMA box per chunk),
-// Q̂[:, 384:576] (3 chunks of [128 x 64]) and P [128 x 64] bf16.
+// Per CTA: TMEM columns [0,256) O half, [256,320) and [320,384) two score buffers S (tile g
+// uses buffer g%2), [384,512) Q̂[:, 0:256] as bf16 pairs (the A operand of the first 16 K-steps
+// of S). The softmax writes P (bf16) over the first 32 columns of its tile's S buffer, and P·C
+// reads it from there (A from TMEM), so a score buffer is free again once P·C of its tile is
+// done: the score MMAs of tile g+1 run while the softmax of tile g works, and the tensor pipe
+// does not wait for it. Shared memory: 2 stages x 9 chunks of [64 tokens x 64 dims] (the whole
+// 576-wide page, 128-byte swizzle, one TMA box per chunk), Q̂[:, 256:576] (5 chunks of
+// [128 x 64]) and the barriers and row maxima (227 KB in all, no alignment slack: the dynamic
+// shared memory starts 1024-byte aligned, which the kernel checks).
+//
+// Shared memory bandwidth, not the tensor pipe, sets the pace on B200: an A-from-smem N = 64
+// K-step reads 6 KB and takes 48 cycles (128 B/clock), an A-from-TMEM one reads 2 KB and
+// takes the MMA's own 32. Per tile a CTA moves ~256 KB through shared memory (72 KB of TMA
+// writes, 152 KB of score operands, 32 KB of P·C operands), ~2000 cycles.
 //
 // Each stage is released in two parts: the 5 chunks only the score MMA reads (the other half's
 // c_KV and k_R) as soon as S is computed, the 4 chunks of this CTA's c_KV half after P·C. The
 // score MMA consumes the early chunks first, so the late chunks' load latency hides behind it.
 //
 // Warp roles (352 threads): warp 0 TMA producer, warp 1 issues the score MMAs, warp 6 issues
-// the P·C MMAs (the two streams get their own warps; each warp stays converged and issues
-// through elect.sync, which on B200 keeps the issue rate at ~37 cycles per N = 64 MMA even
-// while the softmax warps are busy; each accumulator has a single issuer, which keeps the
-// summation order, and the result, deterministic). Warps 2..5 and 7..10 run the softmax,
-// rescale and epilogue: warp w owns TMEM lanes 32*(w%4).. (query rows), and the two warps of a
-// lane quarter split each row's 64 scores (columns 0..31 and 32..63), agreeing on the row
-// maximum through shared memory once per tile.
+// the P·C MMAs (each warp stays converged and issues through elect.sync; each accumulator has
+// a single issuer, which keeps the summation order, and the result, deterministic). Warps
+// 2..5 and 7..10 run the softmax, rescale and epilogue: warp w owns TMEM lanes 32*(w%4)..
+// (query rows), and the two warps of a lane quarter split each row's 64 scores (columns 0..31
+// and 32..63), agreeing on the row maximum through shared memory once per tile.
 // Online softmax in base 2 with a lazy rescale: the running maximum only moves (and O is
 // rescaled) when a new score exceeds it by more than 2^8, which keeps every P <= 256.
 #pragma once
@@ -51,15 +59,13 @@ constexpr int ATT_CHUNK_BYTES = ATT_PAGE * 128;   // [64 rows x 64 bf16]
 constexpr int ATT_CHUNKS = ATT_ROW / 64;          // 9
 constexpr int ATT_TILE_BYTES = ATT_CHUNKS * ATT_CHUNK_BYTES;
 constexpr int ATT_STAGES = 2;
-constexpr int ATT_QT_ELEMS = 384;                 // Q̂ columns kept in TMEM
-constexpr int ATT_QS_CHUNKS = (ATT_ROW - ATT_QT_ELEMS) / 64;   // 3 chunks of Q̂ in smem
+constexpr int ATT_QT_ELEMS = 256;                 // Q̂ columns kept in TMEM
+constexpr int ATT_QT_CHUNKS = ATT_QT_ELEMS / 64;  // 4
+constexpr int ATT_QS_CHUNKS = (ATT_ROW - ATT_QT_ELEMS) / 64;   // 5 chunks of Q̂ in smem
 constexpr int ATT_QS_CHUNK_BYTES = 128 * 128;     // [128 rows x 64 bf16]
-constexpr int ATT_P_BYTES = 128 * 128;            // P [128 x 64] bf16
 constexpr int ATT_THREADS = 352;
 constexpr int ATT_SM_WARPS = 8;                   // softmax warps: 2 per TMEM lane quarter
-constexpr int ATT_SMEM_BYTES =
-    ATT_STAGES * ATT_TILE_BYTES + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES + ATT_P_BYTES + 1024;
-constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 320;
+constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;   // score buffer b at TM_S + 64*b
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;     // log2 units
 
 struct AttnSeg {
@@ -259,13 +265,19 @@ __device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
 struct AttnShared {
   uint64_t full_qk[ATT_STAGES], full_own[ATT_STAGES];    // stage chunks landed (TMA)
   uint64_t empty_qk[ATT_STAGES], empty_own[ATT_STAGES];  // stage chunks free again (MMA commit)
-  uint64_t q_full, q_free, s_full, s_free, p_full, pv_done, o_free, drain;
+  uint64_t s_full[2], p_full[2], pv_done[2];             // per score buffer (tile parity)
+  uint64_t q_full, q_free, o_free, drain;
   uint64_t pair_bar[4];            // the two softmax warps of a lane quarter meet here
-  float row_max[2][2][128];        // [tile parity][column half][row] partial row maxima
-  float row_sum[2][128];           // [column half][row] partial row sums of a segment
+  // [tile parity][column half][row] partial row maxima; a segment's partial row sums reuse
+  // the slot of the parity after its last tile
+  float row_max[2][2][128];
   uint32_t tmem_base;
   volatile int abort_flag;
 };
+
+constexpr int ATT_SMEM_BYTES = ATT_STAGES * ATT_TILE_BYTES + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES +
+                               static_cast<int>(sizeof(AttnShared));
+static_assert(ATT_SMEM_BYTES <= 227 * 1024, "attention kernel exceeds the shared memory of a CTA");
 
 __device__ __forceinline__ bool att_wait(AttnShared& sh, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
@@ -314,13 +326,14 @@ struct TileCursor {
 // The score MMA consumes a tile's chunks in two parts: first the 5 chunks only it needs (the
 // other half's 4 c_KV chunks, then k_R = chunk 8), then this CTA's own 4 c_KV chunks.
 
-// Score K-steps over a run of consecutive chunks c .. c+n-1 of a tile. In the A-from-TMEM form
-// (chunks below 6: Q̂[:, 0:384] sits in TMEM) and the A-from-smem form (Q̂[:, 384:576]). Each
-// run is a short loop whose descriptors only step by constants: the issuing warp shares the
-// instruction cache with the producer, P·C and softmax code (a fully unrolled tile costs more
-// overall), and per-chunk index arithmetic or branching measured ~20 cycles per MMA.
-__device__ __forceinline__ void att_qk_ts(uint32_t tmem, uint64_t b_stage, int c, int n,
-                                          bool first) {
+// Score K-steps over a run of consecutive chunks c .. c+n-1 of a tile into the score buffer at
+// TMEM column d_s. In the A-from-TMEM form (chunks 0..3: Q̂[:, 0:256] sits in TMEM) and the
+// A-from-smem form (chunks 4..8, Q̂[:, 256:576]). Each run is a short loop whose descriptors
+// only step by constants: the issuing warp shares the instruction cache with the producer, P·C
+// and softmax code (a fully unrolled tile costs more overall), and per-chunk index arithmetic
+// or branching measured ~20 cycles per MMA.
+__device__ __forceinline__ void att_qk_ts(uint32_t tmem, uint32_t d_s, uint64_t b_stage, int c,
+                                          int n, bool first) {
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
   uint64_t b0 = b_stage + static_cast<uint64_t>((c * ATT_CHUNK_BYTES) >> 4);
   uint32_t a0 = tmem + TM_Q + c * 32;
@@ -328,58 +341,58 @@ __device__ __forceinline__ void att_qk_ts(uint32_t tmem, uint64_t b_stage, int c
   for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += 32) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts_elect(tmem + TM_S, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
+      mma_bf16_ts_elect(tmem + d_s, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
                         (first && i == 0 && kk == 0) ? 0u : 1u);
   }
 }
-__device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
-                                          int c, int n) {
+__device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint32_t d_s, uint64_t b_stage,
+                                          uint64_t qs_desc, int c, int n, bool first) {
   constexpr uint32_t IDESC_QK = idesc_bf16(128, 64, false, false);
   uint64_t b0 = b_stage + static_cast<uint64_t>((c * ATT_CHUNK_BYTES) >> 4);
   uint64_t a0 =
-      qs_desc + static_cast<uint64_t>(((c - ATT_QT_ELEMS / 64) * ATT_QS_CHUNK_BYTES) >> 4);
+      qs_desc + static_cast<uint64_t>(((c - ATT_QT_CHUNKS) * ATT_QS_CHUNK_BYTES) >> 4);
 #pragma unroll 1
   for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += ATT_QS_CHUNK_BYTES >> 4) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ss_elect(tmem + TM_S, a0 + static_cast<uint64_t>(kk * 2),
-                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK, 1u);
+      mma_bf16_ss_elect(tmem + d_s, a0 + static_cast<uint64_t>(kk * 2),
+                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
+                        (first && i == 0 && kk == 0) ? 0u : 1u);
   }
 }
-// The score-only chunks of a tile: half 0 reads chunks 4,5 | 6,7,8,
-// half 1 chunks 0..3 | 8; the tile's first K-step overwrites S.
-__device__ __forceinline__ void att_qk_score_only(uint32_t tmem, uint64_t b_stage,
+// The score-only chunks of a tile: half 0 reads chunks 4..7 | 8, half 1 chunks 0..3 | 8; the
+// tile's first K-step overwrites S.
+__device__ __forceinline__ void att_qk_score_only(uint32_t tmem, uint32_t d_s, uint64_t b_stage,
                                                   uint64_t qs_desc, int half) {
   if (half == 0) {
-    att_qk_ts(tmem, b_stage, 4, 2, true);
-    att_qk_ss(tmem, b_stage, qs_desc, 6, 3);
+    att_qk_ss(tmem, d_s, b_stage, qs_desc, 4, 5, true);
   } else {
-    att_qk_ts(tmem, b_stage, 0, 4, true);
-    att_qk_ss(tmem, b_stage, qs_desc, 8, 1);
+    att_qk_ts(tmem, d_s, b_stage, 0, 4, true);
+    att_qk_ss(tmem, d_s, b_stage, qs_desc, 8, 1, false);
   }
 }
-// This CTA's own chunks: half 0 chunks 0..3, half 1 chunks 4,5 | 6,7.
-__device__ __forceinline__ void att_qk_own(uint32_t tmem, uint64_t b_stage, uint64_t qs_desc,
-                                           int half) {
-  if (half == 0) {
-    att_qk_ts(tmem, b_stage, 0, 4, false);
-  } else {
-    att_qk_ts(tmem, b_stage, 4, 2, false);
-    att_qk_ss(tmem, b_stage, qs_desc, 6, 2);
-  }
+// This CTA's own chunks: half 0 chunks 0..3, half 1 chunks 4..7.
+__device__ __forceinline__ void att_qk_own(uint32_t tmem, uint32_t d_s, uint64_t b_stage,
+                                           uint64_t qs_desc, int half) {
+  if (half == 0) att_qk_ts(tmem, d_s, b_stage, 0, 4, false);
+  else att_qk_ss(tmem, d_s, b_stage, qs_desc, 4, 4, false);
 }
 
 __global__ void __launch_bounds__(ATT_THREADS, 1)
 mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                        const __grid_constant__ CUtensorMap map_cache4,
                        const __grid_constant__ CUtensorMap map_qhat, AttnParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                             ~static_cast<uintptr_t>(1023));
+  // no static shared memory: the dynamic buffer starts at the CTA's (1024-byte aligned) shared
+  // window, which the 128-byte swizzle of the TMA boxes and MMA descriptors needs
+  extern __shared__ __align__(1024) uint8_t smem[];
+  if ((smem_addr(smem) & 1023u) != 0) {   // uniform over the CTA: nothing has started yet
+    if (threadIdx.x == 0) record_error(MLA_ERR_UNSUPPORTED);
+    return;
+  }
   uint8_t* stage_buf = smem;   // chunk c of stage s at stage_buf + s*TILE + c*CHUNK
   uint8_t* qs_buf = smem + ATT_STAGES * ATT_TILE_BYTES;
-  uint8_t* p_buf = qs_buf + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES;
-  __shared__ AttnShared sh;
+  AttnShared& sh =
+      *reinterpret_cast<AttnShared*>(qs_buf + ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int pair = blockIdx.x >> 1, half = blockIdx.x & 1;
@@ -391,12 +404,13 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
       mbar_init(&sh.empty_qk[s], 1);
       mbar_init(&sh.empty_own[s], 2);   // both MMA threads read a stage's own chunks
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.s_full[b], 1);
+      mbar_init(&sh.p_full[b], ATT_SM_WARPS);
+      mbar_init(&sh.pv_done[b], 1);
+    }
     mbar_init(&sh.q_full, 1 + ATT_SM_WARPS);
     mbar_init(&sh.q_free, 1);
-    mbar_init(&sh.s_full, 1);
-    mbar_init(&sh.s_free, ATT_SM_WARPS);
-    mbar_init(&sh.p_full, ATT_SM_WARPS);
-    mbar_init(&sh.pv_done, 1);
     mbar_init(&sh.o_free, ATT_SM_WARPS);
     mbar_init(&sh.drain, 2);
     for (int q = 0; q < 4; ++q) mbar_init(&sh.pair_bar[q], 2);
@@ -516,19 +530,21 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         TileCursor cur;
         cur.init(p.segs, seg_begin, seg_end);
         for (int g = 0; cur.valid(); ++g, cur.next()) {
-          const int st = g % ATT_STAGES;
+          const int st = g % ATT_STAGES, sb = g & 1;
+          const uint32_t d_s = TM_S + 64 * sb;
           if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) break;
-          if (g >= 1 && !att_warp_wait(sh, &sh.s_free, (g - 1) & 1)) break;
+          // score buffer sb held P of tile g-2: free once P·C of that tile is done
+          if (g >= 2 && !att_warp_wait(sh, &sh.pv_done[sb], ((g >> 1) - 1) & 1)) break;
           const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
           // S over the score-only chunks first, then this CTA's own chunks
           if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          att_qk_score_only(tmem, b_stage, qs_desc, half);
+          att_qk_score_only(tmem, d_s, b_stage, qs_desc, half);
           mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
           if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
           tc_fence_after_sync();
-          att_qk_own(tmem, b_stage, qs_desc, half);
-          mma_commit_elect(&sh.s_full);
+          att_qk_own(tmem, d_s, b_stage, qs_desc, half);
+          mma_commit_elect(&sh.s_full[sb]);
           if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
           mma_commit_elect(&sh.empty_own[st]);
         }
@@ -542,24 +558,25 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         // =========================================================== P·C MMA issuer
         constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
         const uint32_t stage0 = smem_addr(stage_buf);
-        const uint64_t p_desc = smem_desc_sw128(smem_addr(p_buf), 16, 1024);
         TileCursor cur;
         cur.init(p.segs, seg_begin, seg_end);
         for (int g = 0; cur.valid(); ++g, cur.next()) {
-          const int st = g % ATT_STAGES;
+          const int st = g % ATT_STAGES, sb = g & 1;
           const bool first = cur.first_of_seg();
           if (first && cur.k >= 1 && !att_warp_wait(sh, &sh.o_free, (cur.k - 1) & 1)) break;
-          if (!att_warp_wait(sh, &sh.p_full, g & 1)) break;
+          if (!att_warp_wait(sh, &sh.p_full[sb], (g >> 1) & 1)) break;
           tc_fence_after_sync();
-          // O_half += P · C[:, own half]: chunks 4*half .. 4*half+3, read MN-major (N = 256)
+          // O_half += P · C[:, own half]: P (bf16 pairs) from the tile's score buffer in TMEM,
+          // chunks 4*half .. 4*half+3 of the stage read MN-major (N = 256)
           const uint64_t b0 = smem_desc_sw128(
               stage0 + st * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES, ATT_CHUNK_BYTES, 1024);
+          const uint32_t a_p = tmem + TM_S + 64 * sb;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 16 tokens per K-step
-            mma_bf16_ss_elect(tmem + TM_O, p_desc + static_cast<uint64_t>(kk * 2),
-                        b0 + static_cast<uint64_t>(kk * 128), IDESC_PV, (first && kk == 0) ? 0u : 1u);
+          for (int kk = 0; kk < 4; ++kk)   // 16 tokens (8 TMEM columns of P) per K-step
+            mma_bf16_ts_elect(tmem + TM_O, a_p + kk * 8, b0 + static_cast<uint64_t>(kk * 128),
+                              IDESC_PV, (first && kk == 0) ? 0u : 1u);
           mma_commit_elect(&sh.empty_own[st]);
-          mma_commit_elect(&sh.pv_done);
+          mma_commit_elect(&sh.pv_done[sb]);
         }
         mma_commit_elect(&sh.drain);
         if (lane == 0) (void)mbar_wait(&sh.drain, 0);
@@ -583,8 +600,8 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         ++xc;
         return r;
       };
-      // Q̂[:, 0:384] of a unit into TMEM (row r_local), zeros for rows past the unit; each warp
-      // of the pair writes 3 of the 6 column groups.
+      // Q̂[:, 0:256] of a unit into TMEM (row r_local), zeros for rows past the unit; each warp
+      // of the pair writes 2 of the 4 column groups.
       auto load_q_tmem = [&](const AttnSeg& sg) {
         const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
         const int r_in = mt * 128 + r_local;
@@ -593,7 +610,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
             p.qhat + (static_cast<int64_t>(b) * p.R + r_in) * ATT_ROW);
         uint32_t v[32];
 #pragma unroll 1
-        for (int c = hc * 3; c < hc * 3 + 3; ++c) {
+        for (int c = hc * (ATT_QT_CHUNKS / 2); c < (hc + 1) * (ATT_QT_CHUNKS / 2); ++c) {
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const uint4 x = valid ? src[c * 8 + j] : make_uint4(0, 0, 0, 0);
@@ -620,14 +637,14 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         visible_keys(p.keys, b, L, p.Tq, min(p.Tq - 1, (mt * 128 + 127) / p.H), &unused, &hi_u);
         float m_ref = -INFINITY, l_part = 0.0f;
         for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
-          if (!att_warp_wait(sh, &sh.s_full, g & 1)) { ok = false; break; }
+          const int sb = g & 1;
+          const uint32_t s_col = TM_S + 64 * sb;
+          if (!att_warp_wait(sh, &sh.s_full[sb], (g >> 1) & 1)) { ok = false; break; }
           tc_fence_after_sync();
           uint32_t sr[32];
-          tmem_ld32(tmem + t_lane + TM_S + hc * 32, sr);
+          tmem_ld32(tmem + t_lane + s_col + hc * 32, sr);
           tmem_ld_wait();
-          tc_fence_before_sync();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.s_free);
+          tc_fence_before_sync();   // the partner's P store into these columns follows the meeting
           // this thread's visible columns: c_lo .. c_hi of its 32 (none if c_lo > c_hi)
           const int j0 = tile * ATT_PAGE + hc * 32;
           const int c_lo = max(0, lo_row - j0), c_hi = min(31, hi_row - j0);
@@ -647,9 +664,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                                                                  : -INFINITY);
             }
           }
-          // agree on the row maximum with the partner warp (same rows, other 32 columns)
+          // agree on the row maximum with the partner warp (same rows, other 32 columns); after
+          // this meeting both warps hold their S columns in registers, so P may overwrite S
           sh.row_max[g & 1][hc][r_local] = fmaxf(mx0, mx1);
           if (!meet()) { ok = false; break; }
+          tc_fence_after_sync();
           const float raw_max = fmaxf(sh.row_max[g & 1][0][r_local], sh.row_max[g & 1][1][r_local]);
           const float mt_max = raw_max > -INFINITY ? raw_max * p.scale_log2 : -INFINITY;
           float factor = 1.0f;
@@ -663,8 +682,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
               rescale = true;
             }
           }
-          // previous PV must be done before P is overwritten or O is rescaled
-          if (g >= 1 && !att_warp_wait(sh, &sh.pv_done, (g - 1) & 1)) { ok = false; break; }
+          // P·C of the previous tile must be done before O is rescaled
+          if (g >= 1 && !att_warp_wait(sh, &sh.pv_done[(g - 1) & 1], ((g - 1) >> 1) & 1)) {
+            ok = false;
+            break;
+          }
           tc_fence_after_sync();
           if (__any_sync(0xffffffffu, rescale) && tile > sg.tile_begin) {
 #pragma unroll 1
@@ -679,32 +701,27 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
             tmem_st_wait();
           }
           l_part *= factor;
-          // P = 2^(scale*s - m_ref) -> bf16 (0 for hidden columns), this thread's 4 16-byte
-          // chunks of row r_local of the swizzled K-major P tile
+          // P = 2^(scale*s - m_ref) -> bf16 (0 for hidden columns): this thread's 32 keys of row
+          // r_local as 16 bf16 pairs over TMEM columns hc*16.. of the tile's score buffer (key
+          // j of the tile in column j/2, the even key in the low half), the A operand of P·C
           const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
           const float sc = p.scale_log2;
           float ps0 = 0.0f, ps1 = 0.0f;
-          uint8_t* prow = p_buf + r_local * 128;
+          uint32_t w[16];
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t w[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = q * 8 + 2 * e;
-              float x0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
-              float x1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
-              if (!all_vis) {
-                x0 = (c >= c_lo && c <= c_hi) ? x0 : 0.0f;
-                x1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? x1 : 0.0f;
-              }
-              ps0 += x0;
-              ps1 += x1;
-              w[e] = pack_bf16x2(x0, x1);
+          for (int e = 0; e < 16; ++e) {
+            const int c = 2 * e;
+            float x0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
+            float x1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
+            if (!all_vis) {
+              x0 = (c >= c_lo && c <= c_hi) ? x0 : 0.0f;
+              x1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? x1 : 0.0f;
             }
-            const int ch = hc * 4 + q;
-            *reinterpret_cast<uint4*>(prow + ((ch ^ (r_local & 7)) * 16)) =
-                make_uint4(w[0], w[1], w[2], w[3]);
+            ps0 += x0;
+            ps1 += x1;
+            w[e] = pack_bf16x2(x0, x1);
           }
+          tmem_st16(tmem + t_lane + s_col + hc * 16, w);
           l_part += ps0 + ps1;
           // rows outside the keys any row of the unit sees must be zero in the value chunks
           // (P is 0 there, but stale slots past the sequence end, or slots outside a key range,
@@ -723,10 +740,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
                   make_uint4(0, 0, 0, 0);
             }
           }
+          tmem_st_wait();
           fence_proxy_async_smem();
           tc_fence_before_sync();
           __syncwarp();
-          if (lane == 0) mbar_arrive(&sh.p_full);
+          if (lane == 0) mbar_arrive(&sh.p_full[sb]);
         }
         if (!ok) break;
         const int seg_last_g = g - 1;
@@ -736,11 +754,20 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           tc_fence_after_sync();
           load_q_tmem(p.segs[s_i + 1]);
         }
-        // segment epilogue: O / l (this thread's 128 of the CTA's 256 columns) and the lse
-        sh.row_sum[hc][r_local] = l_part;
+        // segment epilogue: O / l (this thread's 128 of the CTA's 256 columns) and the lse. The
+        // partial sums go through the row-maximum slot of the other tile parity: the partner
+        // read its last maxima (tile seg_last_g - 1) before the meeting of tile seg_last_g,
+        // which this warp has passed; a second meeting after the sums are read keeps the next
+        // tile's maxima out of the slot until both warps hold l_sum.
+        float (*row_sum)[128] = sh.row_max[(seg_last_g + 1) & 1];
+        row_sum[hc][r_local] = l_part;
         if (!meet()) { ok = false; break; }
-        const float l_sum = sh.row_sum[0][r_local] + sh.row_sum[1][r_local];
-        if (!att_warp_wait(sh, &sh.pv_done, seg_last_g & 1)) { ok = false; break; }
+        const float l_sum = row_sum[0][r_local] + row_sum[1][r_local];
+        if (!meet()) { ok = false; break; }
+        if (!att_warp_wait(sh, &sh.pv_done[seg_last_g & 1], (seg_last_g >> 1) & 1)) {
+          ok = false;
+          break;
+        }
         tc_fence_after_sync();
         const float inv_l = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
         __nv_bfloat16* dst =
