@@ -17,6 +17,12 @@ __device__ __forceinline__ void record_error(int code) {
   atomicCAS(&g_device_error, 0, code);
 }
 
+// Position of unit (b, mt) (sequence b, 128-row query tile mt) in the split-KV planner's unit
+// stream, which lists every sequence's tile 0, then every sequence's tile 1, ... (B sequences).
+__host__ __device__ __forceinline__ int unit_stream_pos(int b, int mt, int B) {
+  return mt * B + b;
+}
+
 // ------------------------------------------------------------------------- element traits
 
 template <typename T> struct Elem;

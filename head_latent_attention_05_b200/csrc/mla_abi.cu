@@ -789,7 +789,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     const mla_status s = launch_pdl(merge_partials_kernel, dim3((rows + 3) / 4), dim3(256), 0, st,
                                     static_cast<const __nv_bfloat16*>(L.o_part),
                                     static_cast<const float*>(L.lse),
-                                    static_cast<const int32_t*>(L.unit_seg), rows, L.R, L.n_mt,
+                                    static_cast<const int32_t*>(L.unit_seg), rows, L.R,
                                     static_cast<__nv_bfloat16*>(part_out), lse_out);
     mark(3);
     return s;

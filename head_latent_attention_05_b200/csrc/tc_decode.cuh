@@ -33,10 +33,11 @@
 // c_KV and k_R) as soon as S is computed, the 4 chunks of this CTA's c_KV half after P·C. The
 // score MMA consumes the early chunks first, so the late chunks' load latency hides behind it.
 //
-// Warp roles (352 threads): warp 0 TMA producer, warp 1 issues the score MMAs, warp 6 issues
-// the P·C MMAs (each warp stays converged and issues through elect.sync; each accumulator has
-// a single issuer, which keeps the summation order, and the result, deterministic). Warps
-// 2..5 and 7..10 run the softmax, rescale and epilogue: warp w owns TMEM lanes 32*(w%4)..
+// Warp roles (320 threads): warp 0 TMA producer, warp 1 issues every MMA (S of a tile, then
+// P·C of the tile before; it stays converged and issues through elect.sync; a single issuer
+// keeps the summation order, and the result, deterministic). A second issuing warp for P·C
+// measured ~200 ns per tcgen05 instruction on B200 against ~36 ns in the score warp. Warps
+// 2..5 and 6..9 run the softmax, rescale and epilogue: warp w owns TMEM lanes 32*(w%4)..
 // (query rows), and the two warps of a lane quarter split each row's 64 scores (columns 0..31
 // and 32..63), agreeing on the row maximum through shared memory once per tile.
 // Online softmax in base 2 with a lazy rescale: the running maximum only moves (and O is
@@ -63,7 +64,7 @@ constexpr int ATT_QT_ELEMS = 256;                 // Q̂ columns kept in TMEM
 constexpr int ATT_QT_CHUNKS = ATT_QT_ELEMS / 64;  // 4
 constexpr int ATT_QS_CHUNKS = (ATT_ROW - ATT_QT_ELEMS) / 64;   // 5 chunks of Q̂ in smem
 constexpr int ATT_QS_CHUNK_BYTES = 128 * 128;     // [128 rows x 64 bf16]
-constexpr int ATT_THREADS = 352;
+constexpr int ATT_THREADS = 320;
 constexpr int ATT_SM_WARPS = 8;                   // softmax warps: 2 per TMEM lane quarter
 constexpr uint32_t TM_O = 0, TM_S = 256, TM_Q = 384;   // score buffer b at TM_S + 64*b
 constexpr float ATT_RESCALE_THRESHOLD = 8.0f;     // log2 units
@@ -95,9 +96,9 @@ struct PlanParams {
   const int32_t* seq_lens;
   int B, Tq, H, n_mt, max_pos, P, max_segs;
   KeyRange keys;
-  int32_t* unit_first;   // [U] scratch: first page of each unit's key range
-  int32_t* unit_tiles;   // [U] scratch: first global tile of each unit
-  int32_t* unit_seg;     // [U + 1]
+  int32_t* unit_first;   // [U] scratch: first page of each unit's key range (by stream position)
+  int32_t* unit_tiles;   // [U] scratch: first virtual tile of each unit (by stream position)
+  int32_t* unit_seg;     // [U + 1] first segment of each unit (by stream position)
   int32_t* pair_seg;     // [P + 1]
   AttnSeg* segs;         // [max_segs]
 };
@@ -157,6 +158,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* excl, int* warp_
 // holding the last key its last token sees (visible_keys: causal, window, key range), so a
 // prefill's early tokens and a windowed decode skip the pages none of their rows can see.
 //
+// Order. Units are laid out in the stream query-tile major: position i = mt * B + b holds
+// unit (b, mt) (unit_stream_pos). The units of one sequence cover nearly the same pages, so
+// cutting this stream into equal ranges gives the pairs of every query tile the same relative
+// position in their part: pair j of tile 0 and pair j of tile 1 stream the same pages at the
+// same time, and the second read of each page comes from L2 instead of HBM. Everything the
+// planner writes per unit (unit_first, unit_tiles, unit_seg) is indexed by stream position;
+// a segment's `unit` field holds the unit itself, b * n_mt + mt.
+//
 // Balance. A CTA pair pays a fixed price each time it moves on to another unit (the finished
 // segment's epilogue and the next unit's Q̂ load lie on its critical path; measured at about
 // five tiles' worth on B200). So the tile list is cut in a virtual stream in which every unit
@@ -172,14 +181,14 @@ __device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
   constexpr int C = ATT_SEG_COST_TILES;
   const int U = pp.B * pp.n_mt;
   const int nt = static_cast<int>(blockDim.x);
-  // pass 1: tiles per unit -> virtual unit starts
+  // pass 1: tiles per unit -> virtual unit starts (u: stream position)
   if (threadIdx.x == 0) carry_s = 0;
   __syncthreads();
   for (int u0 = 0; u0 < U; u0 += nt) {
     const int u = u0 + threadIdx.x;
     int n = 0;
     if (u < U) {
-      const int b = u / pp.n_mt, mt = u % pp.n_mt;
+      const int b = u % pp.B, mt = u / pp.B;
       const int L = pp.seq_lens[b];
       int first = 0;
       if (L >= pp.Tq && L <= pp.max_pos) {
@@ -236,7 +245,7 @@ __device__ __noinline__ void attn_plan_block(const PlanParams& pp) {
         const int e = min(v1, ps[p + 1]);
         if (e <= a) continue;
         AttnSeg sg;
-        sg.unit = u;
+        sg.unit = (u % pp.B) * pp.n_mt + u / pp.B;
         sg.tile_begin = pp.unit_first[u] + (a - v0);
         sg.tile_end = pp.unit_first[u] + (e - v0);
         sg.pair = p;
@@ -402,7 +411,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
       mbar_init(&sh.full_qk[s], 1);
       mbar_init(&sh.full_own[s], 1);
       mbar_init(&sh.empty_qk[s], 1);
-      mbar_init(&sh.empty_own[s], 2);   // both MMA threads read a stage's own chunks
+      mbar_init(&sh.empty_own[s], 2);   // the own chunks' score MMAs and P·C both commit
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.s_full[b], 1);
@@ -412,7 +421,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
     mbar_init(&sh.q_full, 1 + ATT_SM_WARPS);
     mbar_init(&sh.q_free, 1);
     mbar_init(&sh.o_free, ATT_SM_WARPS);
-    mbar_init(&sh.drain, 2);
+    mbar_init(&sh.drain, 1);
     for (int q = 0; q < 4; ++q) mbar_init(&sh.pair_bar[q], 2);
     sh.abort_flag = 0;
     fence_mbar_init();
@@ -523,69 +532,71 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
       }
     } else if (warp == 1) {
       {
-        // =========================================================== score MMA issuer
-        // (the whole warp runs this loop; one elected lane issues each MMA and commit)
-        const uint32_t stage0 = smem_addr(stage_buf);
-        const uint64_t qs_desc = smem_desc_sw128(smem_addr(qs_buf), 16, 1024);
-        TileCursor cur;
-        cur.init(p.segs, seg_begin, seg_end);
-        for (int g = 0; cur.valid(); ++g, cur.next()) {
-          const int st = g % ATT_STAGES, sb = g & 1;
-          const uint32_t d_s = TM_S + 64 * sb;
-          if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) break;
-          // score buffer sb held P of tile g-2: free once P·C of that tile is done
-          if (g >= 2 && !att_warp_wait(sh, &sh.pv_done[sb], ((g >> 1) - 1) & 1)) break;
-          const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
-          // S over the score-only chunks first, then this CTA's own chunks
-          if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) break;
-          tc_fence_after_sync();
-          att_qk_score_only(tmem, d_s, b_stage, qs_desc, half);
-          mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
-          if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
-          tc_fence_after_sync();
-          att_qk_own(tmem, d_s, b_stage, qs_desc, half);
-          mma_commit_elect(&sh.s_full[sb]);
-          if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
-          mma_commit_elect(&sh.empty_own[st]);
-        }
-        // drain: every MMA issued above completes before TMEM is released
-        mma_commit_elect(&sh.drain);
-        if (lane == 0) (void)mbar_wait(&sh.drain, 0);
-        __syncwarp();
-      }
-    } else if (warp == 6) {
-      {   // the whole warp runs this loop; one elected lane issues
-        // =========================================================== P·C MMA issuer
+        // ======================================== MMA issuer: S of tile g, then P·C of g-1
+        // (the whole warp runs this loop; one elected lane issues each MMA and commit). One
+        // warp issues both streams in this order: S(g) needs only P·C(g-2) done (its score
+        // buffer), and the softmax of g-1 overlaps S(g); P·C(g-1) follows as soon as P(g-1)
+        // is in TMEM. (Issuing P·C(g-1) between the two parts of S(g) measured no faster: the
+        // tensor pipe runs its queue in order.)
         constexpr uint32_t IDESC_PV = idesc_bf16(128, 256, false, true);
         const uint32_t stage0 = smem_addr(stage_buf);
-        TileCursor cur;
-        cur.init(p.segs, seg_begin, seg_end);
-        for (int g = 0; cur.valid(); ++g, cur.next()) {
-          const int st = g % ATT_STAGES, sb = g & 1;
-          const bool first = cur.first_of_seg();
-          if (first && cur.k >= 1 && !att_warp_wait(sh, &sh.o_free, (cur.k - 1) & 1)) break;
-          if (!att_warp_wait(sh, &sh.p_full[sb], (g >> 1) & 1)) break;
+        const uint64_t qs_desc = smem_desc_sw128(smem_addr(qs_buf), 16, 1024);
+        // O_half += P · C[:, own half] for tile gv: P (bf16 pairs) from the tile's score buffer
+        // in TMEM, chunks 4*half .. 4*half+3 of its stage read MN-major (N = 256); the first
+        // tile of a segment (k-th of this CTA) overwrites O once the last epilogue has read it
+        auto issue_pv = [&](int gv, bool first_v, int kv) -> bool {
+          const int st = gv % ATT_STAGES, sb = gv & 1;
+          if (first_v && kv >= 1 && !att_warp_wait(sh, &sh.o_free, (kv - 1) & 1)) return false;
+          if (!att_warp_wait(sh, &sh.p_full[sb], (gv >> 1) & 1)) return false;
           tc_fence_after_sync();
-          // O_half += P · C[:, own half]: P (bf16 pairs) from the tile's score buffer in TMEM,
-          // chunks 4*half .. 4*half+3 of the stage read MN-major (N = 256)
           const uint64_t b0 = smem_desc_sw128(
               stage0 + st * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES, ATT_CHUNK_BYTES, 1024);
           const uint32_t a_p = tmem + TM_S + 64 * sb;
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)   // 16 tokens (8 TMEM columns of P) per K-step
             mma_bf16_ts_elect(tmem + TM_O, a_p + kk * 8, b0 + static_cast<uint64_t>(kk * 128),
-                              IDESC_PV, (first && kk == 0) ? 0u : 1u);
+                              IDESC_PV, (first_v && kk == 0) ? 0u : 1u);
           mma_commit_elect(&sh.empty_own[st]);
           mma_commit_elect(&sh.pv_done[sb]);
+          return true;
+        };
+        TileCursor cur;
+        cur.init(p.segs, seg_begin, seg_end);
+        bool ok = true, prev_first = false;
+        int g = 0, prev_k = 0;
+        for (; cur.valid(); ++g, cur.next()) {
+          const int st = g % ATT_STAGES, sb = g & 1;
+          const uint32_t d_s = TM_S + 64 * sb;
+          if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) { ok = false; break; }
+          // score buffer sb held P of tile g-2: free once P·C of that tile is done
+          if (g >= 2 && !att_warp_wait(sh, &sh.pv_done[sb], ((g >> 1) - 1) & 1)) { ok = false; break; }
+          const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);
+          // S over the score-only chunks first, then this CTA's own chunks
+          if (!att_warp_wait(sh, &sh.full_qk[st], (g / ATT_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after_sync();
+          att_qk_score_only(tmem, d_s, b_stage, qs_desc, half);
+          mma_commit_elect(&sh.empty_qk[st]);   // arrives once these MMAs have read their chunks
+          if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) { ok = false; break; }
+          tc_fence_after_sync();
+          att_qk_own(tmem, d_s, b_stage, qs_desc, half);
+          mma_commit_elect(&sh.s_full[sb]);
+          if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
+          mma_commit_elect(&sh.empty_own[st]);
+          if (g >= 1 && !issue_pv(g - 1, prev_first, prev_k)) { ok = false; break; }
+          prev_first = cur.first_of_seg();
+          prev_k = cur.k;
         }
+        if (ok && g >= 1) (void)issue_pv(g - 1, prev_first, prev_k);
+        // drain: every MMA issued above completes before TMEM is released
         mma_commit_elect(&sh.drain);
         if (lane == 0) (void)mbar_wait(&sh.drain, 0);
         __syncwarp();
       }
     } else {
       // ============================================================ softmax warps
-      // Warps 2..5 take score columns 0..31, warps 7..10 columns 32..63 of the same rows.
-      const int hc = warp >= 7 ? 1 : 0;   // column half of the score tile
+      // Warps 2..5 take score columns 0..31, warps 6..9 columns 32..63 of the same rows (each
+      // group covers the four TMEM lane quarters, warp w reading lanes 32*(w%4)..).
+      const int hc = warp >= 6 ? 1 : 0;   // column half of the score tile
       const int quarter = warp & 3;
       const int r_local = quarter * 32 + lane;
       const int t_idx = hc * 128 + r_local;   // 0..255 among the softmax threads

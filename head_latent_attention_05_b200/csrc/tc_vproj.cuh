@@ -23,7 +23,8 @@ namespace mla {
 struct VprojParams {
   const __nv_bfloat16* o_part;  // partial O / l (bf16), see above
   const float* lse;             // their log-sum-exp, see above
-  const int32_t* unit_seg;      // [U + 1] first segment of each unit (segment mode)
+  const int32_t* unit_seg;      // [U + 1] first segment of each unit by stream position
+                                //   (unit_stream_pos; segment mode)
   __nv_bfloat16* out;           // [n_q][H][d_v]
   int H, Tq, n_mt, n_q, d_v;
   int n_parts;                  // 0: segment mode
@@ -101,7 +102,7 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
       } else {
         const int b = n / p.Tq, t = n % p.Tq;
         const int r = t * p.H + h;
-        const int u = b * p.n_mt + r / 128;
+        const int u = unit_stream_pos(b, r / 128, p.n_q / p.Tq);
         const int s0 = p.unit_seg[u];
         base[ps] = static_cast<int64_t>(s0) * 128 + r % 128;
         cnt[ps] = p.unit_seg[u + 1] - s0;
@@ -240,14 +241,14 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
 // Rows are row = n * H + h (n = b * Tq + t); 64 threads per row, 8 dims each, 4 rows a block.
 __global__ void __launch_bounds__(256)
 merge_partials_kernel(const __nv_bfloat16* __restrict__ o_seg, const float* __restrict__ lse_seg,
-                      const int32_t* __restrict__ unit_seg, int rows, int R, int n_mt,
+                      const int32_t* __restrict__ unit_seg, int rows, int R,
                       __nv_bfloat16* __restrict__ o_out, float* __restrict__ lse_out) {
   pdl_wait();
   const int row = blockIdx.x * 4 + static_cast<int>(threadIdx.x >> 6);
   const int k = threadIdx.x & 63;
   if (row >= rows) return;
   const int b = row / R, r_in = row % R;
-  const int u = b * n_mt + r_in / 128, rl = r_in % 128;
+  const int u = unit_stream_pos(b, r_in / 128, rows / R), rl = r_in % 128;
   const int s0 = unit_seg[u], s1 = unit_seg[u + 1];
   float mx = -INFINITY;
   for (int s = s0; s < s1; ++s) mx = fmaxf(mx, lse_seg[static_cast<int64_t>(s) * 128 + rl]);
