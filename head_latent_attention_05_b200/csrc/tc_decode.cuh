@@ -347,12 +347,8 @@ __device__ __forceinline__ void att_qk_ts(uint32_t tmem, uint32_t d_s, uint64_t 
   uint64_t b0 = b_stage + static_cast<uint64_t>((c * ATT_CHUNK_BYTES) >> 4);
   uint32_t a0 = tmem + TM_Q + c * 32;
 #pragma unroll 1
-  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += 32) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ts_elect(tmem + d_s, a0 + kk * 8, b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
-                        (first && i == 0 && kk == 0) ? 0u : 1u);
-  }
+  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += 32)
+    mma_bf16_ts_x4_elect(tmem + d_s, a0, b0, IDESC_QK, (first && i == 0) ? 0u : 1u);
 }
 __device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint32_t d_s, uint64_t b_stage,
                                           uint64_t qs_desc, int c, int n, bool first) {
@@ -361,13 +357,8 @@ __device__ __forceinline__ void att_qk_ss(uint32_t tmem, uint32_t d_s, uint64_t 
   uint64_t a0 =
       qs_desc + static_cast<uint64_t>(((c - ATT_QT_CHUNKS) * ATT_QS_CHUNK_BYTES) >> 4);
 #pragma unroll 1
-  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += ATT_QS_CHUNK_BYTES >> 4) {
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16_ss_elect(tmem + d_s, a0 + static_cast<uint64_t>(kk * 2),
-                        b0 + static_cast<uint64_t>(kk * 2), IDESC_QK,
-                        (first && i == 0 && kk == 0) ? 0u : 1u);
-  }
+  for (int i = 0; i < n; ++i, b0 += ATT_CHUNK_BYTES >> 4, a0 += ATT_QS_CHUNK_BYTES >> 4)
+    mma_bf16_ss_x4_elect(tmem + d_s, a0, b0, IDESC_QK, (first && i == 0) ? 0u : 1u);
 }
 // The score-only chunks of a tile: half 0 reads chunks 4..7 | 8, half 1 chunks 0..3 | 8; the
 // tile's first K-step overwrites S.
@@ -663,9 +654,9 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           float mx0 = -INFINITY, mx1 = -INFINITY;
           if (all_vis) {
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-              mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-              mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+            for (int c = 0; c < 32; c += 4) {
+              mx0 = fmax3(mx0, __uint_as_float(sr[c]), __uint_as_float(sr[c + 1]));
+              mx1 = fmax3(mx1, __uint_as_float(sr[c + 2]), __uint_as_float(sr[c + 3]));
             }
           } else {
 #pragma unroll
@@ -715,24 +706,31 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           // P = 2^(scale*s - m_ref) -> bf16 (0 for hidden columns): this thread's 32 keys of row
           // r_local as 16 bf16 pairs over TMEM columns hc*16.. of the tile's score buffer (key
           // j of the tile in column j/2, the even key in the low half), the A operand of P·C
+          // (pairs of columns in f32x2 arithmetic: the even and odd columns' exponent arguments
+          // and partial sums, each lane rounded as its scalar form would be)
           const float neg_m = (m_ref == -INFINITY) ? 0.0f : -m_ref;
           const float sc = p.scale_log2;
-          float ps0 = 0.0f, ps1 = 0.0f;
+          const uint64_t sc2 = f2_pack(sc, sc), nm2 = f2_pack(neg_m, neg_m);
+          uint64_t ps2 = f2_pack(0.0f, 0.0f);
           uint32_t w[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int c = 2 * e;
-            float x0 = fast_exp2(fmaf(__uint_as_float(sr[c]), sc, neg_m));
-            float x1 = fast_exp2(fmaf(__uint_as_float(sr[c + 1]), sc, neg_m));
+            float x0, x1;
+            f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2),
+                      x0, x1);
+            x0 = fast_exp2(x0);
+            x1 = fast_exp2(x1);
             if (!all_vis) {
               x0 = (c >= c_lo && c <= c_hi) ? x0 : 0.0f;
               x1 = (c + 1 >= c_lo && c + 1 <= c_hi) ? x1 : 0.0f;
             }
-            ps0 += x0;
-            ps1 += x1;
+            ps2 = f2_add(ps2, f2_pack(x0, x1));
             w[e] = pack_bf16x2(x0, x1);
           }
           tmem_st16(tmem + t_lane + s_col + hc * 16, w);
+          float ps0, ps1;
+          f2_unpack(ps2, ps0, ps1);
           l_part += ps0 + ps1;
           // rows outside the keys any row of the unit sees must be zero in the value chunks
           // (P is 0 there, but stale slots past the sequence end, or slots outside a key range,
