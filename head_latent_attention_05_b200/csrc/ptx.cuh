@@ -226,6 +226,25 @@ __device__ __forceinline__ void mma_bf16_ts_x4_elect(uint32_t d_tmem, uint32_t a
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first)
       : "memory");
 }
+// Four K = 16 steps of an MN-major B operand (P·C): A from TMEM columns a_tmem + 8*kk, B
+// descriptor b_desc + 128*kk (16 rows of 128 bytes further along K).
+__device__ __forceinline__ void mma_bf16_ts_mn_x4_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                        uint64_t b_desc, uint32_t idesc,
+                                                        uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, t, e;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a1, a2, a3;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.s64 b1, %2, 128;\n\tadd.s64 b2, %2, 256;\n\tadd.s64 b3, %2, 384;\n\t"
+      "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a1], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a2], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [a3], b3, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first)
+      : "memory");
+}
 // The same with A from shared memory: A descriptor a_desc + 2*kk.
 __device__ __forceinline__ void mma_bf16_ss_x4_elect(uint32_t d_tmem, uint64_t a_desc,
                                                      uint64_t b_desc, uint32_t idesc,

@@ -402,7 +402,7 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
       mbar_init(&sh.full_qk[s], 1);
       mbar_init(&sh.full_own[s], 1);
       mbar_init(&sh.empty_qk[s], 1);
-      mbar_init(&sh.empty_own[s], 2);   // the own chunks' score MMAs and P·C both commit
+      mbar_init(&sh.empty_own[s], 1);   // committed after the stage's P·C
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.s_full[b], 1);
@@ -543,10 +543,9 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           const uint64_t b0 = smem_desc_sw128(
               stage0 + st * ATT_TILE_BYTES + half * 4 * ATT_CHUNK_BYTES, ATT_CHUNK_BYTES, 1024);
           const uint32_t a_p = tmem + TM_S + 64 * sb;
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)   // 16 tokens (8 TMEM columns of P) per K-step
-            mma_bf16_ts_elect(tmem + TM_O, a_p + kk * 8, b0 + static_cast<uint64_t>(kk * 128),
-                              IDESC_PV, (first_v && kk == 0) ? 0u : 1u);
+          // 4 K-steps of 16 tokens (8 TMEM columns of P, 16 rows of the chunks)
+          mma_bf16_ts_mn_x4_elect(tmem + TM_O, a_p, b0, IDESC_PV, first_v ? 0u : 1u);
+          // (tracks every earlier MMA of this thread: the stage's own chunks are free after it)
           mma_commit_elect(&sh.empty_own[st]);
           mma_commit_elect(&sh.pv_done[sb]);
           return true;
@@ -572,7 +571,6 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           att_qk_own(tmem, d_s, b_stage, qs_desc, half);
           mma_commit_elect(&sh.s_full[sb]);
           if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
-          mma_commit_elect(&sh.empty_own[st]);
           if (g >= 1 && !issue_pv(g - 1, prev_first, prev_k)) { ok = false; break; }
           prev_first = cur.first_of_seg();
           prev_k = cur.k;
