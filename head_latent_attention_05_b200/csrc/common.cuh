@@ -125,18 +125,26 @@ struct RopeFreqs {
 // are within 1 of an even integer, or are even integers themselves), and sinpi/cospi take the
 // small remainder. Everything stays in fp32 (fp64 is slow on the device), and for positions up
 // to 2^30 the angle keeps an absolute error of about 1e-6 rad.
-__device__ __forceinline__ void rope_pair(float x, float y, float f_hi, float f_lo, int pos,
-                                          float* ox, float* oy) {
+__device__ __forceinline__ void rope_sincos(float f_hi, float f_lo, int pos, float* s, float* c) {
   const float a = static_cast<float>(pos & ~0xFFF), b = static_cast<float>(pos & 0xFFF);
   const float p1 = a * f_hi, e1 = fmaf(a, f_hi, -p1);
   const float p2 = b * f_hi, e2 = fmaf(b, f_hi, -p2);
   const float r1 = p1 - 2.0f * rintf(0.5f * p1);
   const float r2 = p2 - 2.0f * rintf(0.5f * p2);
   const float t = (r1 + r2) + ((e1 + e2) + fmaf(a, f_lo, b * f_lo));
+  sincospif(t, s, c);
+}
+// The turn itself, (x, y) -> (x cos - y sin, x sin + y cos), with explicit fused rounding so
+// that every caller rounds alike.
+__device__ __forceinline__ void rope_turn(float x, float y, float s, float c, float* ox, float* oy) {
+  *ox = fmaf(x, c, -(y * s));
+  *oy = fmaf(x, s, y * c);
+}
+__device__ __forceinline__ void rope_pair(float x, float y, float f_hi, float f_lo, int pos,
+                                          float* ox, float* oy) {
   float s, c;
-  sincospif(t, &s, &c);
-  *ox = x * c - y * s;
-  *oy = x * s + y * c;
+  rope_sincos(f_hi, f_lo, pos, &s, &c);
+  rope_turn(x, y, s, c, ox, oy);
 }
 
 }  // namespace mla

@@ -6,6 +6,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -741,18 +742,22 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     const uint64_t db[3] = {static_cast<uint64_t>(qrow), static_cast<uint64_t>(H),
                             static_cast<uint64_t>(n_q)};
     const uint64_t sb[2] = {static_cast<uint64_t>(qrow) * 2, static_cast<uint64_t>(qrow) * 2 * H};
-    // at most 128 tokens per CTA: 4 accumulators of bn columns fill TMEM's 512, and the ring
-    // plus the RoPE box stay within shared memory
+    // at most 128 tokens per CTA: 4 accumulators of bn columns fill TMEM's 512
     const int bn = pick_bn(n_q) > 128 ? 128 : pick_bn(n_q);
     const uint32_t bb[3] = {64, 1, static_cast<uint32_t>(bn)};
     if (!make_map(&mA, w_uk_t, 3, da, sa, ba) || !make_map(&mB, q, 3, db, sb, bb))
       return MLA_ERR_CUDA;
     const int m_per_cta = ATT_DC / 128;
-    GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1, m_per_cta, 1};
+    // q_rope turns: one thread per (token, rotary pair), at most 16 blocks (the SMs the H head
+    // CTAs leave free)
+    const int rope_items = n_q * (ATT_DR / 2);
+    const int rope_blocks = std::min(16, (rope_items + 127) / 128);
+    GemmShape shp{ATT_DC, n_q, cfg->d_nope / 64, cfg->d_nope / 64, 1, 1, m_per_cta,
+                  1 + rope_blocks};
     PlanParams pp{seq_lens, batch, tq, H, L.n_mt, max_pos, L.P, L.max_segs, keys,
                   L.unit_first, L.unit_tiles, L.unit_seg, L.pair_seg, L.segs};
     EpiQhat epi{L.qhat, static_cast<const __nv_bfloat16*>(q), seq_lens, H, tq, ATT_DC, ATT_DR,
-                cfg->d_nope, n_q, max_pos, bn, pp, rope_freqs(cfg)};
+                cfg->d_nope, n_q, max_pos, rope_blocks, pp, rope_freqs(cfg)};
     const mla_status s = launch_gemm(mA, mB, shp, ATT_DC / 128, H, epi, st, bn);
     if (s != MLA_OK) return s;
   }

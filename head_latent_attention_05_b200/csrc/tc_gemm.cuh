@@ -11,9 +11,13 @@
 //
 // Roles in a 128-thread CTA: warp 0 / lane 0 issues TMA loads, warp 1 allocates TMEM and issues
 // the MMAs (the whole warp runs the loop, one elected lane issues), warps 2-3 run the epilogue
-// functor's side job (Epi::side); afterwards all four warps read D out of TMEM (warp w owns TMEM lanes
-// 32w..32w+31 = rows m0+32w..) and hand each value to the epilogue functor. Extra blocks at the
-// end of grid.z (GemmShape::aux_blocks) skip the GEMM and run the functor's aux() job instead.
+// functor's side job (Epi::side); afterwards all four warps read D out of TMEM (warp w owns TMEM
+// lanes 32w..32w+31 = rows m0+32w..), convert each value to the functor's output type and stage
+// the m-tile in shared memory (the drained load ring) as [token][128 m], so that each token's
+// 128 outputs, contiguous in every output layout used here, leave in 16-byte stores: scattered
+// 2-byte stores (one per thread and token) measured ~85 cycles a warp instruction on B200 and
+// made the epilogue most of the kernel. Extra blocks at the end of grid.z
+// (GemmShape::aux_blocks) skip the GEMM and run the functor's aux() job instead.
 #pragma once
 
 #include "common.cuh"
@@ -63,8 +67,9 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   constexpr uint32_t IDESC = idesc_bf16(128, BN, false, false);
 
   if (static_cast<int>(blockIdx.z) >= static_cast<int>(gridDim.z) - shp.aux_blocks) {
-    // the aux slice of grid.z exists for every (x, y); its job runs once
-    if (blockIdx.x == 0 && blockIdx.y == 0) epi.aux();
+    // the aux slice of grid.z exists for every (x, y); each of its jobs runs once
+    if (blockIdx.x == 0 && blockIdx.y == 0)
+      epi.aux(static_cast<int>(blockIdx.z) - (static_cast<int>(gridDim.z) - shp.aux_blocks));
     return;
   }
 
@@ -167,24 +172,41 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
   if (ready) (void)mbar_try_wait(&done_bar, 0);
   else if ((threadIdx.x & 31) == 0) record_error(MLA_ERR_DEVICE_TIMEOUT);
+  // block-uniform (every thread has left its role): the staging loop below syncs the block
+  ready = __syncthreads_and(ready ? 1 : 0) != 0;
   tc_fence_after_sync();
   if (ready && nk > 0) {
+    using Out = typename Epi::Out;
+    static_assert(BN * 128 * sizeof(Out) <= STAGES * STAGE_BYTES, "staging tile exceeds the ring");
+    constexpr int VEC = 16 / static_cast<int>(sizeof(Out));   // outputs per 16-byte store
+    constexpr int ROW_VECS = 128 / VEC;
+    Out* stage = reinterpret_cast<Out*>(smem);   // [BN][128]; every load and MMA has completed
 #pragma unroll 1
     for (int mt = 0; mt < n_mt; ++mt) {
-      const int m = (mt0 + mt) * 128 + threadIdx.x;
+      const int m_base = (mt0 + mt) * 128;
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_at(tmem, warp * 32, mt * BN + c0), v);
         tmem_ld_wait();
-        if (m < shp.M) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + c0 + j;
-            if (n < shp.N) epi(z, split, m, n, __uint_as_float(v[j]));
-          }
+        for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + threadIdx.x] = Epi::cvt(__uint_as_float(v[j]));
+      }
+      __syncthreads();
+      const int m_rows = min(128, shp.M - m_base);
+      for (int i = threadIdx.x; i < BN * ROW_VECS; i += blockDim.x) {
+        const int nl = i / ROW_VECS, mv = (i % ROW_VECS) * VEC;
+        const int n = n0 + nl;
+        if (n >= shp.N || mv >= m_rows) continue;
+        Out* dst = epi.row(z, split, n) + m_base + mv;
+        const Out* src = stage + nl * 128 + mv;
+        if (mv + VEC <= m_rows && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+        } else {
+          for (int e = 0; e < VEC && mv + e < m_rows; ++e) dst[e] = src[e];
         }
       }
+      __syncthreads();   // the next m-tile reuses the staging tile
     }
   }
   tc_fence_before_sync();
@@ -198,19 +220,24 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
 
 // ------------------------------------------------------------------------------ epilogues
 
+// Output interface of every functor: Out (the stored type), cvt (fp32 accumulator -> Out) and
+// row(z, split, n), the address of output (m = 0, n); a row's m outputs are contiguous.
+
 // Append down-projection with split-K: partial[split][n][m] (fp32), summed later in order.
 struct EpiSplitK {
   float* partial;
   int n_tok, F;
+  using Out = float;
+  __device__ static float cvt(float v) { return v; }
+  __device__ float* row(int, int split, int n) const {
+    return partial + (static_cast<int64_t>(split) * n_tok + n) * F;
+  }
   struct SideState {};
   __host__ __device__ static constexpr int side_bytes(int) { return 0; }
-  __device__ void aux() const {}
+  __device__ void aux(int) const {}
   __device__ SideState side_begin(int, int, int) const { return {}; }
   __device__ void side_issue(const CUtensorMap*, uint8_t*, uint64_t*, int, int) const {}
   __device__ void side(int, int, int, int, int, const SideState&, const uint8_t*, uint64_t*) const {}
-  __device__ void operator()(int, int split, int m, int n, float v) const {
-    partial[(static_cast<int64_t>(split) * n_tok + n) * F + m] = v;
-  }
 };
 
 // Plain store: out[n][m] = v rounded to bf16, rows of `ld` elements (the q path's up-projection
@@ -218,89 +245,80 @@ struct EpiSplitK {
 struct EpiStoreBf16 {
   __nv_bfloat16* out;
   int ld;
+  using Out = __nv_bfloat16;
+  __device__ static __nv_bfloat16 cvt(float v) { return __float2bfloat16_rn(v); }
+  __device__ __nv_bfloat16* row(int, int, int n) const { return out + static_cast<int64_t>(n) * ld; }
   struct SideState {};
   __host__ __device__ static constexpr int side_bytes(int) { return 0; }
-  __device__ void aux() const {}
+  __device__ void aux(int) const {}
   __device__ SideState side_begin(int, int, int) const { return {}; }
   __device__ void side_issue(const CUtensorMap*, uint8_t*, uint64_t*, int, int) const {}
   __device__ void side(int, int, int, int, int, const SideState&, const uint8_t*, uint64_t*) const {}
-  __device__ void operator()(int, int, int m, int n, float v) const {
-    out[static_cast<int64_t>(n) * ld + m] = __float2bfloat16_rn(v);
-  }
 };
 
-// Absorbed query: qhat[(n*H + h)][m] = q_lat (bf16), m < d_c. Warps 2-3 of the n-tile-0 CTA of
-// head h also write the rotated rope part qhat[..][d_c + i] while the MMAs run, and the one aux
-// block runs the split-KV planner of the attention kernel that follows.
+// Absorbed query: qhat[(n*H + h)][m] = q_lat (bf16), m < d_c. Aux block 0 runs the split-KV
+// planner of the attention kernel that follows; aux blocks 1..rope_blocks write the rotated rope
+// part qhat[..][d_c:] (rope_rows) while the head CTAs stream W_UK.
 struct EpiQhat {
   __nv_bfloat16* qhat;
   const __nv_bfloat16* q;        // [B*Tq][H][d_nope + d_r]
   const int32_t* seq_lens;       // [B]
   int H, Tq, d_c, d_r, d_nope, n_rows, max_pos;
-  int box_rows;                  // tokens per CTA (the GEMM's BN)
+  int rope_blocks;               // aux blocks that rotate q_rope (after the planner's one)
   PlanParams plan;
   RopeFreqs rope;
-  __device__ void aux() const { attn_plan_block(plan); }
-  // RoPE(q_rope) of head h for this CTA's BN tokens, written to qhat[..][d_c:] by warps 2-3 of
-  // the m-tile-0 CTA while the MMAs run. The producer brings the BN x 64 q_rope box in with the
-  // B tensor map (128-byte swizzle) ahead of the weight stream; each side thread owns one token
-  // (the token's length is read at the start, before the stream begins) and a share of its
-  // rotary pairs.
-  struct SideState {
-    int len;   // seq_lens of the first token this thread handles
-  };
-  __host__ __device__ static constexpr int side_bytes(int bn) { return bn * 128; }
-  __device__ bool rope_cta() const { return blockIdx.x == 0; }
-  __device__ SideState side_begin(int tid, int nt, int n0) const {
-    SideState st{-1};
-    const int t1 = box_rows < nt ? box_rows : nt;
-    const int n = n0 + tid % t1;
-    if (rope_cta() && n < n_rows) st.len = seq_lens[n / Tq];
-    return st;
+  using Out = __nv_bfloat16;
+  __device__ static __nv_bfloat16 cvt(float v) { return __float2bfloat16_rn(v); }
+  __device__ __nv_bfloat16* row(int h, int, int n) const {
+    return qhat + (static_cast<int64_t>(n) * H + h) * (d_c + d_r);
   }
-  __device__ void side_issue(const CUtensorMap* map_q, uint8_t* side_smem, uint64_t* bar, int h,
-                             int n0) const {
-    if (!rope_cta()) return;
-    mbar_arrive_expect_tx(bar, static_cast<uint32_t>(side_box_rows() * 128));
-    tma_load_3d(side_smem, map_q, bar, d_nope, h, n0);
+  struct SideState {};
+  __host__ __device__ static constexpr int side_bytes(int) { return 0; }
+  __device__ SideState side_begin(int, int, int) const { return {}; }
+  __device__ void side_issue(const CUtensorMap*, uint8_t*, uint64_t*, int, int) const {}
+  __device__ void side(int, int, int, int, int, const SideState&, const uint8_t*, uint64_t*) const {}
+  __device__ void aux(int i) const {
+    if (i == 0) attn_plan_block(plan);
+    else rope_rows(i - 1);
   }
-  __device__ int side_box_rows() const { return box_rows; }
-  __device__ void side(int h, int, int tid, int nt, int n0, const SideState& st,
-                       const uint8_t* side_smem, uint64_t* bar) const {
-    if (!rope_cta()) return;
-    const int lane = tid & 31;
-    bool ok = true;
-    if (lane == 0) ok = mbar_wait(bar, 0);
-    if (__shfl_sync(0xffffffffu, ok ? 1 : 0, 0) == 0) {
-      if (lane == 0) record_error(MLA_ERR_DEVICE_TIMEOUT);
-      return;
-    }
-    (void)mbar_try_wait(bar, 0);
-    const int row = d_c + d_r;
-    const int half = d_r / 2;                    // 32 pairs, one 128-byte smem row per token
-    const int t1 = box_rows < nt ? box_rows : nt;   // token columns handled at once
-    const int groups = nt / t1;                  // pair groups per token
-    const int pg = tid / t1;
-    for (int nl = tid % t1, first = 1; nl < box_rows; nl += t1, first = 0) {
-      const int n = n0 + nl;
-      if (n >= n_rows) break;
-      const int L = first ? st.len : seq_lens[n / Tq];
-      const bool ok_len = L >= Tq && L <= max_pos;
-      const int ps = L - Tq + n % Tq;
-      for (int r = pg; r < half; r += groups) {
-        // element 2r of row nl in the swizzled box: 16-byte chunk (2r/8) ^ (nl % 8)
-        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(
-            side_smem + nl * 128 + ((((2 * r) >> 3) ^ (nl & 7)) << 4) + ((2 * r) & 7) * 2);
-        float ox = 0.0f, oy = 0.0f;
-        if (ok_len)
-          rope_pair(__low2float(v), __high2float(v), rope.f_hi[r], rope.f_lo[r], ps, &ox, &oy);
-        *reinterpret_cast<__nv_bfloat162*>(qhat + (static_cast<int64_t>(n) * H + h) * row + d_c +
-                                           2 * r) = __floats2bfloat162_rn(ox, oy);
+  // RoPE(q_rope) of every (token, head). The angle depends on the token's position and the pair
+  // only, so one thread per (token, pair) computes it once and turns that pair for all H heads;
+  // a warp covers 32 pairs of one token, i.e. 128 contiguous bytes of a (token, head) row per
+  // load and store.
+  __device__ void rope_rows(int blk) const {
+    const int half = d_r / 2;
+    const int qrow = d_nope + d_r, orow = d_c + d_r;   // elements per (token, head) row
+    const int64_t total = static_cast<int64_t>(n_rows) * half;
+    const int64_t step = static_cast<int64_t>(rope_blocks) * blockDim.x;
+    for (int64_t idx = static_cast<int64_t>(blk) * blockDim.x + threadIdx.x; idx < total;
+         idx += step) {
+      const int n = static_cast<int>(idx / half), r = static_cast<int>(idx % half);
+      const int L = seq_lens[n / Tq];
+      const bool ok = L >= Tq && L <= max_pos;
+      float sn = 0.0f, cs = 0.0f;
+      if (ok) rope_sincos(rope.f_hi[r], rope.f_lo[r], L - Tq + n % Tq, &sn, &cs);
+      const __nv_bfloat162* src = reinterpret_cast<const __nv_bfloat162*>(
+          q + static_cast<int64_t>(n) * H * qrow + d_nope) + r;
+      __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(
+          qhat + static_cast<int64_t>(n) * H * orow + d_c) + r;
+      // 32 heads' loads in flight at a time (the rows come from HBM: latency, not bandwidth)
+      constexpr int HB = 32;
+      for (int h0 = 0; h0 < H; h0 += HB) {
+        __nv_bfloat162 v[HB];
+#pragma unroll
+        for (int j = 0; j < HB; ++j)
+          v[j] = h0 + j < H ? src[static_cast<int64_t>(h0 + j) * (qrow / 2)]
+                            : __floats2bfloat162_rn(0.0f, 0.0f);
+#pragma unroll
+        for (int j = 0; j < HB; ++j) {
+          if (h0 + j >= H) break;
+          const float2 f = __bfloat1622float2(v[j]);
+          float ox = 0.0f, oy = 0.0f;
+          if (ok) rope_turn(f.x, f.y, sn, cs, &ox, &oy);
+          dst[static_cast<int64_t>(h0 + j) * (orow / 2)] = __floats2bfloat162_rn(ox, oy);
+        }
       }
     }
-  }
-  __device__ void operator()(int h, int, int m, int n, float v) const {
-    qhat[(static_cast<int64_t>(n) * H + h) * (d_c + d_r) + m] = __float2bfloat16_rn(v);
   }
 };
 

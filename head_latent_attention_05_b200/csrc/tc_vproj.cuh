@@ -111,49 +111,63 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
   }
   pdl_wait();   // the attention partials are complete and visible from here on
   pdl_trigger();
+  // thread k of a row holds the lse of the row's segment k (rows rarely have more than TPR
+  // segments; later ones are read where needed), every pass's load in flight at once; the
+  // other threads of the row take it by shuffle, so each pass waits for one round of partial
+  // loads only
+  float lse_k[PASSES];
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps)
+    lse_k[ps] = k < cnt[ps] ? p.lse[base[ps] + k * stride] * lse_scale : -INFINITY;
 #pragma unroll
   for (int ps = 0; ps < PASSES; ++ps) {
     const int rr = ps * RP + rr_l;
     const int s1 = cnt[ps];
     const int64_t rb = base[ps];
     auto lse_of = [&](int s) { return p.lse[rb + s * stride] * lse_scale; };
-    float mx = -INFINITY;
-    for (int s = k; s < s1; s += TPR) mx = fmaxf(mx, lse_of(s));
+    float mx = lse_k[ps];
+    for (int s = k + TPR; s < s1; s += TPR) mx = fmaxf(mx, lse_of(s));
 #pragma unroll
     for (int o = TPR / 2; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    const bool any = mx > -INFINITY;
     float den = 0.0f;
     float acc[32];
 #pragma unroll
     for (int e = 0; e < 32; ++e) acc[e] = 0.0f;
-    if (mx > -INFINITY) {
-      for (int s = k; s < s1; s += TPR) den += exp2f(lse_of(s) - mx);
-      // four partials' loads in flight at a time; the sum runs in partial order
-      for (int sb = 0; sb < s1; sb += 4) {
-        float w[4];
-        uint4 v[4][4];
+    if (any) {
+      if (k < s1) den = exp2f(lse_k[ps] - mx);
+      for (int s = k + TPR; s < s1; s += TPR) den += exp2f(lse_of(s) - mx);
+    }
+    // four partials' loads in flight at a time; the sum runs in partial order. The trip count
+    // is the larger of the warp's two rows (the shuffles need every lane).
+    const int s1w = __reduce_max_sync(0xffffffffu, s1);
+    for (int sb = 0; sb < s1w; sb += 4) {
+      float w[4];
+      uint4 v[4][4];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const int s = sb + j;
-          w[j] = 0.0f;
-          if (s < s1) {
-            w[j] = exp2f(lse_of(s) - mx);
-            const uint4* src = reinterpret_cast<const uint4*>(p.o_part + (rb + s * stride) * ATT_DC);
+      for (int j = 0; j < 4; ++j) {
+        const int s = sb + j;
+        float ls = __shfl_sync(0xffffffffu, lse_k[ps], s & (TPR - 1), TPR);
+        w[j] = 0.0f;
+        if (any && s < s1) {
+          if (s >= TPR) ls = lse_of(s);
+          w[j] = exp2f(ls - mx);
+          const uint4* src = reinterpret_cast<const uint4*>(p.o_part + (rb + s * stride) * ATT_DC);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) v[j][i] = src[k + TPR * i];
-          }
+          for (int i = 0; i < 4; ++i) v[j][i] = src[k + TPR * i];
         }
+      }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          if (sb + j >= s1) break;
+      for (int j = 0; j < 4; ++j) {
+        if (!any || sb + j >= s1) break;
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const uint32_t u[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t u[4] = {v[j][i].x, v[j][i].y, v[j][i].z, v[j][i].w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
-              acc[8 * i + 2 * e] = fmaf(w[j], f.x, acc[8 * i + 2 * e]);
-              acc[8 * i + 2 * e + 1] = fmaf(w[j], f.y, acc[8 * i + 2 * e + 1]);
-            }
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u[e]));
+            acc[8 * i + 2 * e] = fmaf(w[j], f.x, acc[8 * i + 2 * e]);
+            acc[8 * i + 2 * e + 1] = fmaf(w[j], f.y, acc[8 * i + 2 * e + 1]);
           }
         }
       }
@@ -198,30 +212,45 @@ vproj_merge_kernel(const __grid_constant__ CUtensorMap map_wuv, VprojParams p) {
   }
   __syncwarp();
 
-  // ---- epilogue: warps 0..3, thread = row m0 + threadIdx.x of the d_v tile
+  // ---- epilogue: warps 0..3 (thread = row m0 + threadIdx.x of the d_v tile) stage D as
+  // [token][128] bf16 in the B operand buffer (its MMAs are done), then all threads store each
+  // (token, head) row's 128 outputs in 16-byte pieces (one 2-byte store per thread and token
+  // measured far slower)
+  bool ready = true;
   if (warp < 4) {
-    bool ready = false;
+    ready = false;
     if (lane == 0) ready = mbar_wait(&done_bar, 0);
     ready = __shfl_sync(0xffffffffu, ready ? 1 : 0, 0) != 0;
     if (ready) (void)mbar_try_wait(&done_bar, 0);
     else if (lane == 0) record_error(MLA_ERR_DEVICE_TIMEOUT);
-    tc_fence_after_sync();
-    const int m = m0 + threadIdx.x;
-    if (ready) {
+  }
+  ready = __syncthreads_and(ready ? 1 : 0) != 0;   // block-uniform: the stores below sync
+  tc_fence_after_sync();
+  if (ready) {
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(b_buf);
+    if (warp < 4) {
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 16) {
         uint32_t v[16];
         tmem_ld16(tmem_at(tmem, warp * 32, c0), v);
         tmem_ld_wait();
-        if (m < p.d_v) {
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int n = n0 + c0 + j;
-            if (n < p.n_q)
-              p.out[(static_cast<int64_t>(n) * p.H + h) * p.d_v + m] =
-                  __float2bfloat16_rn(__uint_as_float(v[j]));
-          }
-        }
+        for (int j = 0; j < 16; ++j)
+          stage[(c0 + j) * 128 + threadIdx.x] = __float2bfloat16_rn(__uint_as_float(v[j]));
+      }
+    }
+    __syncthreads();
+    const int m_rows = min(128, p.d_v - m0);
+    for (int i = threadIdx.x; i < BN * 16; i += VP_THREADS) {
+      const int nl = i >> 4, mv = (i & 15) * 8;
+      const int n = n0 + nl;
+      if (n >= p.n_q || mv >= m_rows) continue;
+      __nv_bfloat16* dst = p.out + (static_cast<int64_t>(n) * p.H + h) * p.d_v + m0 + mv;
+      const __nv_bfloat16* src = stage + nl * 128 + mv;
+      if (mv + 8 <= m_rows && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
+        *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
+      } else {
+        for (int e = 0; e < 8 && mv + e < m_rows; ++e) dst[e] = src[e];
       }
     }
   }
