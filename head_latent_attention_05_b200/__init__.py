@@ -66,6 +66,16 @@ def make_config(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size=64, dtype=
 _lib = None
 
 
+def use_library(path: str) -> None:
+    """Load the C ABI from another build of the same sources (e.g. the short-wait test build)
+    for the calls that follow; use_library(LIB_PATH) goes back to the product library. Each
+    library keeps its own device error word."""
+    global LIB_PATH, _lib
+    LIB_PATH = path
+    _lib = None
+    load_library()
+
+
 def load_library() -> ctypes.CDLL:
     """Load libmla.so from the package directory; raise if it is missing."""
     global _lib

@@ -3,6 +3,9 @@
 //
 // Every wait here is bounded: it gives up after MLA_WAIT_TIMEOUT_NS of wall time (read from
 // %globaltimer) and returns false, so a kernel can record MLA_ERR_DEVICE_TIMEOUT and leave.
+// The attention kernel's pipeline waits take MLA_PIPE_WAIT_NS (the same by default); its
+// drains, which wait for copies and MMAs already in flight before the CTA may exit, keep the
+// long limit. A test build shortens only the pipeline limit to exercise the abort path.
 #pragma once
 
 #include <cstdint>
@@ -12,6 +15,9 @@
 
 #ifndef MLA_WAIT_TIMEOUT_NS
 #define MLA_WAIT_TIMEOUT_NS 2000000000ull   // 2 s
+#endif
+#ifndef MLA_PIPE_WAIT_NS
+#define MLA_PIPE_WAIT_NS MLA_WAIT_TIMEOUT_NS
 #endif
 
 namespace mla {

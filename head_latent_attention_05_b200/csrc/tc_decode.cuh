@@ -275,7 +275,9 @@ struct AttnShared {
   uint64_t full_qk[ATT_STAGES], full_own[ATT_STAGES];    // stage chunks landed (TMA)
   uint64_t empty_qk[ATT_STAGES], empty_own[ATT_STAGES];  // stage chunks free again (MMA commit)
   uint64_t s_full[2], p_full[2], pv_done[2];             // per score buffer (tile parity)
-  uint64_t q_full, q_free, o_free, drain;
+  uint64_t q_full;                 // the softmax warps wrote a unit's Q̂[:, 0:256] into TMEM
+  uint64_t qs_full;                // the unit's Q̂[:, 256:576] landed in shared memory (TMA)
+  uint64_t q_free, o_free, drain;
   uint64_t pair_bar[4];            // the two softmax warps of a lane quarter meet here
   // [tile parity][column half][row] partial row maxima; a segment's partial row sums reuse
   // the slot of the parity after its last tile
@@ -294,7 +296,7 @@ __device__ __forceinline__ bool att_wait(AttnShared& sh, uint64_t* bar, uint32_t
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (sh.abort_flag) return false;
-    if (global_timer_ns() - t0 > MLA_WAIT_TIMEOUT_NS) {
+    if (global_timer_ns() - t0 > MLA_PIPE_WAIT_NS) {
       sh.abort_flag = 1;
       record_error(MLA_ERR_DEVICE_TIMEOUT);
       return false;
@@ -409,7 +411,8 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
       mbar_init(&sh.p_full[b], ATT_SM_WARPS);
       mbar_init(&sh.pv_done[b], 1);
     }
-    mbar_init(&sh.q_full, 1 + ATT_SM_WARPS);
+    mbar_init(&sh.q_full, ATT_SM_WARPS);
+    mbar_init(&sh.qs_full, 1);
     mbar_init(&sh.q_free, 1);
     mbar_init(&sh.o_free, ATT_SM_WARPS);
     mbar_init(&sh.drain, 1);
@@ -458,12 +461,14 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           if (!own)
             tma_load_2d(st + 8 * ATT_CHUNK_BYTES, &map_cache, bar, 64 * 8, page * ATT_PAGE);
         };
-        auto load_q_smem = [&](const AttnSeg& sg) {   // Q̂[:, 384:576] of a unit
+        int n_qloads = 0;   // Q̂ loads issued: the last one is drained before the CTA leaves
+        auto load_q_smem = [&](const AttnSeg& sg) {   // Q̂[:, 256:576] of a unit
           const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
-          mbar_arrive_expect_tx(&sh.q_full, ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES);
+          mbar_arrive_expect_tx(&sh.qs_full, ATT_QS_CHUNKS * ATT_QS_CHUNK_BYTES);
           for (int c = 0; c < ATT_QS_CHUNKS; ++c)
-            tma_load_2d(qs_buf + c * ATT_QS_CHUNK_BYTES, &map_qhat, &sh.q_full,
+            tma_load_2d(qs_buf + c * ATT_QS_CHUNK_BYTES, &map_qhat, &sh.qs_full,
                         ATT_QT_ELEMS + 64 * c, b * p.R + mt * 128);
+          ++n_qloads;
         };
         // Step for tile g: its own chunks, then (new segment at g+1) the next Q̂, then the
         // score-only chunks of tile g+1. Own chunks of g wait for P·C of g-2; score-only chunks
@@ -515,7 +520,10 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
           cq.next();
           ++gq;
         }
-        // drain: the last loads must land before the CTA can exit (bounded, abort or not)
+        // drain: the last loads must land before the CTA can exit (bounded, abort or not); a
+        // Q̂ load is issued only after the score MMAs consumed the one before, so only the last
+        // can still be in flight, and likewise for each stage's two rings
+        if (n_qloads > 0) (void)mbar_wait(&sh.qs_full, (n_qloads - 1) & 1);
         for (int j = max(0, gq - ATT_STAGES); j < gq; ++j)
           (void)mbar_wait(&sh.full_qk[j % ATT_STAGES], (j / ATT_STAGES) & 1);
         for (int j = max(0, go - ATT_STAGES); j < go; ++j)
@@ -557,7 +565,11 @@ mla_decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache,
         for (; cur.valid(); ++g, cur.next()) {
           const int st = g % ATT_STAGES, sb = g & 1;
           const uint32_t d_s = TM_S + 64 * sb;
-          if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) { ok = false; break; }
+          if (cur.first_of_seg() && (!att_warp_wait(sh, &sh.q_full, cur.k & 1) ||
+                                     !att_warp_wait(sh, &sh.qs_full, cur.k & 1))) {
+            ok = false;
+            break;
+          }
           // score buffer sb held P of tile g-2: free once P·C of that tile is done
           if (g >= 2 && !att_warp_wait(sh, &sh.pv_done[sb], ((g >> 1) - 1) & 1)) { ok = false; break; }
           const uint64_t b_stage = smem_desc_sw128(stage0 + st * ATT_TILE_BYTES, 16, 1024);

@@ -177,36 +177,61 @@ gemm_tc_kernel(const __grid_constant__ CUtensorMap mapA, const __grid_constant__
   tc_fence_after_sync();
   if (ready && nk > 0) {
     using Out = typename Epi::Out;
-    static_assert(BN * 128 * sizeof(Out) <= STAGES * STAGE_BYTES, "staging tile exceeds the ring");
+    constexpr int TILE = BN * 128;                              // staged outputs per m-tile
+    constexpr int GROUP = (STAGES * STAGE_BYTES) / (TILE * static_cast<int>(sizeof(Out)));
+    static_assert(GROUP >= 1, "staging tile exceeds the ring");
     constexpr int VEC = 16 / static_cast<int>(sizeof(Out));   // outputs per 16-byte store
     constexpr int ROW_VECS = 128 / VEC;
-    Out* stage = reinterpret_cast<Out*>(smem);   // [BN][128]; every load and MMA has completed
+    Out* stage = reinterpret_cast<Out*>(smem);   // [m-tile][BN][128]; loads and MMAs are done
+    // as many m-tiles as the ring holds are staged, then all their rows leave at once
 #pragma unroll 1
-    for (int mt = 0; mt < n_mt; ++mt) {
-      const int m_base = (mt0 + mt) * 128;
+    for (int g0 = 0; g0 < n_mt; g0 += GROUP) {
+      const int g1 = min(n_mt, g0 + GROUP);
 #pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 16) {
-        uint32_t v[16];
-        tmem_ld16(tmem_at(tmem, warp * 32, mt * BN + c0), v);
-        tmem_ld_wait();
+      for (int mt = g0; mt < g1; ++mt) {
+        Out* tile = stage + (mt - g0) * TILE;
+        if constexpr (BN % 64 == 0) {   // 64 columns per wait
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 64) {
+            uint32_t v0[32], v1[32];
+            tmem_ld32(tmem_at(tmem, warp * 32, mt * BN + c0), v0);
+            tmem_ld32(tmem_at(tmem, warp * 32, mt * BN + c0 + 32), v1);
+            tmem_ld_wait();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) stage[(c0 + j) * 128 + threadIdx.x] = Epi::cvt(__uint_as_float(v[j]));
+            for (int j = 0; j < 32; ++j) {
+              tile[(c0 + j) * 128 + threadIdx.x] = Epi::cvt(__uint_as_float(v0[j]));
+              tile[(c0 + 32 + j) * 128 + threadIdx.x] = Epi::cvt(__uint_as_float(v1[j]));
+            }
+          }
+        } else {
+#pragma unroll 1
+          for (int c0 = 0; c0 < BN; c0 += 16) {
+            uint32_t v[16];
+            tmem_ld16(tmem_at(tmem, warp * 32, mt * BN + c0), v);
+            tmem_ld_wait();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) tile[(c0 + j) * 128 + threadIdx.x] = Epi::cvt(__uint_as_float(v[j]));
+          }
+        }
       }
       __syncthreads();
-      const int m_rows = min(128, shp.M - m_base);
-      for (int i = threadIdx.x; i < BN * ROW_VECS; i += blockDim.x) {
-        const int nl = i / ROW_VECS, mv = (i % ROW_VECS) * VEC;
+      const int items = (g1 - g0) * BN * ROW_VECS;
+      for (int i = threadIdx.x; i < items; i += blockDim.x) {
+        const int t = i / (BN * ROW_VECS), rem = i % (BN * ROW_VECS);
+        const int nl = rem / ROW_VECS, mv = (rem % ROW_VECS) * VEC;
         const int n = n0 + nl;
+        const int m_base = (mt0 + g0 + t) * 128;
+        const int m_rows = min(128, shp.M - m_base);
         if (n >= shp.N || mv >= m_rows) continue;
         Out* dst = epi.row(z, split, n) + m_base + mv;
-        const Out* src = stage + nl * 128 + mv;
+        const Out* src = stage + t * TILE + nl * 128 + mv;
         if (mv + VEC <= m_rows && (reinterpret_cast<uintptr_t>(dst) & 15u) == 0) {
           *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(src);
         } else {
           for (int e = 0; e < VEC && mv + e < m_rows; ++e) dst[e] = src[e];
         }
       }
-      __syncthreads();   // the next m-tile reuses the staging tile
+      __syncthreads();   // the next group reuses the staging area
     }
   }
   tc_fence_before_sync();
@@ -301,8 +326,8 @@ struct EpiQhat {
           q + static_cast<int64_t>(n) * H * qrow + d_nope) + r;
       __nv_bfloat162* dst = reinterpret_cast<__nv_bfloat162*>(
           qhat + static_cast<int64_t>(n) * H * orow + d_c) + r;
-      // 32 heads' loads in flight at a time (the rows come from HBM: latency, not bandwidth)
-      constexpr int HB = 32;
+      // 64 heads' loads in flight at a time (the rows come from HBM: latency, not bandwidth)
+      constexpr int HB = 64;
       for (int h0 = 0; h0 < H; h0 += HB) {
         __nv_bfloat162 v[HB];
 #pragma unroll

@@ -23,9 +23,11 @@
  *     they enqueue kernels on `stream` and return. Arguments are validated on the host first:
  *     on any error the call returns a non-zero mla_status and enqueues nothing.
  *   - Errors that only the device can see (a page id outside the pool, a sequence length out
- *     of range, a stalled pipeline) are recorded in the device error word; the affected
- *     outputs are zero-filled, no memory outside the given buffers is touched, and the next
- *     mla_get_device_error call reports the first such error.
+ *     of range, a stalled pipeline) are recorded in the device error word, and the next
+ *     mla_get_device_error call reports the first such error. No memory outside the given
+ *     buffers is touched. A bad page id or length zero-fills the affected outputs; after a
+ *     stalled pipeline (a bounded wait that ran out, MLA_ERR_DEVICE_TIMEOUT) the kernel drains
+ *     its copies and MMAs and leaves, and the call's outputs are undefined.
  *   - Calls that share a workspace or a cache must not overlap on the GPU (use one stream).
  *   - Within a call, kernels after the first are launched with programmatic dependent launch
  *     and let the next kernel of the stream start early. A caller's own kernel enqueued right
