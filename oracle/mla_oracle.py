@@ -328,3 +328,82 @@ def mha_cache_elems_per_token(n_heads: int, d_h: int) -> int:
 def gqa_cache_elems_per_token(n_groups: int, d_h: int) -> int:
     """GQA with n_groups key/value groups: 2·n_groups·d_h."""
     return 2 * n_groups * d_h
+
+
+# --- quantised latent cache (8-bit codes with one scale per token) --------------------------
+#
+# 「Multi-Head Latent Attention（MLA）原理与工程实践全解析」 (context only) quantises the latent
+# per token: one scale for a token's whole latent row. Read here as: every cache row
+# [c_KV | k_R] is stored as FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7, 3 mantissa bits;
+# no infinities, 0x7F/0xFF are NaN; largest finite value 448) plus one float32 scale
+#     scale = max_i |v_i| / 448,   code_i = E4M3(v_i / scale)   (round to nearest, ties to
+# even, saturating at ±448), and the stored row means code_i * scale. A row of zeros gets scale 0.
+# The rounding to E4M3 decides an integer code, so these steps are done in float32, as the
+# device does them (row values arrive as float32): the max is exact, each division is one
+# correctly rounded float32 division, then one rounding onto the E4M3 grid.
+
+E4M3_MAX = 448.0
+
+
+def e4m3_value(code) -> np.ndarray:
+    """Real value of FP8 E4M3 codes (uint8 array), float64; NaN for 0x7F and 0xFF.
+
+    From the format's definition: exponent field e and mantissa m give (1 + m/8)·2^(e-7) for
+    e >= 1 and m/8·2^(-6) for e = 0 (subnormal); e = 15, m = 7 is NaN (the format keeps the
+    rest of the top binade for finite values, up to 1.75·2^8 = 448).
+    """
+    c = np.asarray(code, dtype=np.int64)
+    sign = np.where(c & 0x80, -1.0, 1.0)
+    e = (c >> 3) & 0xF
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e.astype(np.float64) - 7))
+    out = sign * mag
+    return np.where((c & 0x7F) == 0x7F, np.nan, out)
+
+
+_E4M3_GRID = e4m3_value(np.arange(127))   # the non-negative finite values, increasing with code
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Nearest FP8 E4M3 code of each value of x (float64 view of float32 inputs): round to
+    nearest, ties to the even code (even mantissa), magnitudes at or above 448 saturate to
+    ±448, the sign of zero and of values that round to zero is kept (IEEE rounding)."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    hi = np.clip(np.searchsorted(_E4M3_GRID, a, side="left"), 1, 126)   # grid[hi-1] < a <= grid[hi]
+    lo = hi - 1
+    d_lo = a - _E4M3_GRID[lo]
+    d_hi = _E4M3_GRID[hi] - a
+    pick = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(lo % 2 == 0, lo, hi)))
+    pick = np.where(a >= E4M3_MAX, 126, pick)
+    pick = np.where(a == 0.0, 0, pick)
+    neg = np.signbit(x)
+    return (pick | np.where(neg, 0x80, 0)).astype(np.uint8)
+
+
+def quantize_rows_e4m3(rows):
+    """Per-token quantisation of cache rows: rows [n, d] (float32 values) ->
+    (codes uint8 [n, d], scales float32 [n]). Every step in float32, as the device does it."""
+    r = np.asarray(rows, dtype=np.float32)
+    amax = np.max(np.abs(r), axis=-1)
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    safe = np.where(scale > 0, scale, np.float32(1.0)).astype(np.float32)
+    q = (r / safe[..., None]).astype(np.float32)                          # one rounding each
+    codes = e4m3_encode(q.astype(np.float64))
+    return codes, scale
+
+
+def dequantize_rows_e4m3(codes, scales) -> np.ndarray:
+    """The row values a quantised cache stores: code value × the token's scale, float64."""
+    return e4m3_value(codes) * f64(scales)[..., None]
+
+
+def gather_rows_fp8(codes, scales, block_table_row, L: int, page_size: int = 64) -> np.ndarray:
+    """The L dequantised rows of one sequence of a quantised paged cache, read through its
+    block-table row: codes [num_pages, page_size, d], scales [num_pages, page_size]."""
+    idx = np.arange(L)
+    pages = np.asarray(block_table_row, dtype=np.int64)[idx // page_size]
+    slots = idx % page_size
+    c = np.asarray(codes)[pages, slots]
+    s = np.asarray(scales)[pages, slots]
+    return dequantize_rows_e4m3(c, s)
