@@ -46,7 +46,7 @@ METRIC = "MLA decode cache-tokens/s (×heads) on 1 B200; % of HBM/tensor rooflin
 UNIT = "cache_tokens*heads/s"
 DEFAULT_WORKLOAD = "v2_bf16_b64_ctx1kto32k_mix"
 # measured after the headline, each with its own attention roofline
-EXTRA_WORKLOADS = ("v2_bf16_b16_ctx4096", "v2_bf16_b4_ctx131072_tq2")
+EXTRA_WORKLOADS = ("v2_bf16_b16_ctx4096", "v2_bf16_b4_ctx131072_tq2", "v2_fp8_b64_ctx1kto32k_mix")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 ATTN_PROFILE = os.path.join(ROOT, "profiles", "attn_kernel_traffic.json")
 
@@ -56,7 +56,8 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=WL.WORKLOAD_ORDER)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD,
+                    choices=WL.WORKLOAD_ORDER + list(WL.EXTRA_WORKLOADS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="budget of the oracle CPU-baseline sample")
@@ -85,7 +86,8 @@ def work_of(w: WL.Workload, lens: torch.Tensor) -> dict:
     Ls = [int(v) for v in lens.tolist()]
     tokens = sum(Ls)
     elem = 4 if w.dtype == "f32" else 2
-    cache_bytes = tokens * w.row * elem
+    # a quantised cache row: one byte per code plus its float32 scale
+    cache_bytes = tokens * (w.row + 4) if w.kv == "fp8" else tokens * w.row * elem
     w_bytes = 2 * w.H * w.d_nope * w.d_c * elem          # W_UK + W_UV
     attn_flops = sum(L * w.Tq for L in Ls) * w.H * 2 * (w.row + w.d_c)
     proj_flops = 2 * (2 * w.B * w.Tq * w.H * w.d_nope * w.d_c)
@@ -205,7 +207,8 @@ def build_inputs(w: WL.Workload, device):
     lens = WL.seq_lens(w)
     pt = WL.page_table(w, lens)
     weights = WL.weights(w)
-    cache_host = WL.cache_pool(w, pt.num_pages)
+    cache_host = (WL.cache_pool_fp8(w, pt.num_pages) if w.kv == "fp8"
+                  else WL.cache_pool(w, pt.num_pages))
     x_new, seq_idx, pos, q = WL.new_token_inputs(w, lens)
     return lens, pt, weights, cache_host, x_new, seq_idx, pos, q
 
@@ -260,7 +263,7 @@ class DeviceCase:
         (self.lens, self.pt, self.weights, self.cache_host, self.x_new_h, self.seq_idx_h,
          self.pos_h, self.q_h) = build_inputs(w, dev)
         self.cfg = mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, WL.PAGE_SIZE,
-                                   w.dtype, w.scale, w.rms_eps, w.rope_theta)
+                                   w.dtype, w.scale, w.rms_eps, w.rope_theta, kv_format=w.kv)
         dt = w.torch_dtype
         self.cache = self.cache_host.to(dev)
         self.bt = self.pt.block_table.to(dev)
@@ -333,7 +336,7 @@ def attn_roofline(w: WL.Workload, work: dict, t_attn_s: float, ms_per_step: floa
     roof["traffic"] = stored_traffic(w.name)
     roof["peak_source"] = (f"{pk_kind} (MEASURED_PEAKS.json: burst bf16 GEMM, copy HBM)"
                            if pk_kind == "measured" else "fallback")
-    roof["kernel"] = "mla_decode_attn_kernel"
+    roof["kernel"] = "mla_decode_attn_fp8_kernel" if w.kv == "fp8" else "mla_decode_attn_kernel"
     roof["kernel_us"] = t_attn_s * 1e6
     roof["algorithmic_bytes_per_launch"] = work["cache_bytes"]
     roof["algorithmic_flops_per_launch"] = work["attn_flops"]
@@ -518,7 +521,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    w = WL.WORKLOADS[args.workload]
+    w = WL.get(args.workload)
     K, Wm = args.steps, max(3, args.warmup)
     flush_l2 = L2Flush(dev)
     c = DeviceCase(mla, w, dev)
@@ -557,7 +560,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         for name in EXTRA_WORKLOADS:
             if name == w.name:
                 continue
-            ce = DeviceCase(mla, WL.WORKLOADS[name], dev)
+            ce = DeviceCase(mla, WL.get(name), dev)
             me = measure_device(ce, flush_l2, min(K, args.extra_steps), Wm, world,
                                 not args.no_graph, local_rank)
             extra[name] = {"value": me["value"], "unit": UNIT, "ms_per_step": me["ms_per_step"],
@@ -568,7 +571,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             torch.cuda.empty_cache()
         line["other_workloads"] = extra
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kv == "plain":
         lens, pt, weights, cache_host, x_new_h, pos_h, q_h = cpu_case
         threading = ("serial loop over (sequence, head) units; cores = the BLAS thread count that "
                      "numpy's matrix products may use inside one unit")
@@ -593,22 +596,26 @@ def stored_traffic(workload: str):
         return None
     with open(ATTN_PROFILE) as f:
         prof = json.load(f)
-    sha = kernel_sha()
+    sha = kernel_sha(fp8=WL.get(workload).kv == "fp8")
     for e in prof.get("captures", []):
         if e.get("workload") == workload and e.get("kernel_source_sha") == sha:
             return e.get("dram_bytes_per_launch")
     return None
 
 
-def kernel_sha() -> str:
+def kernel_sha(fp8: bool = False) -> str:
     """Hash of the attention kernel's code (its source with // comments and blank lines
-    dropped), to tell whether stored counters are still current."""
+    dropped), to tell whether stored counters are still current. The quantised-cache kernel
+    is hashed together with the file it builds on."""
     import hashlib
     import re
-    path = os.path.join(ROOT, "head_latent_attention_05_b200", "csrc", "tc_decode.cuh")
-    with open(path, encoding="utf-8") as f:
-        lines = [re.sub(r"//.*", "", ln).rstrip() for ln in f]
-    code = "\n".join(ln for ln in lines if ln.strip())
+    files = ["tc_decode.cuh"] + (["tc_decode_fp8.cuh", "fp8_cache.cuh"] if fp8 else [])
+    code = ""
+    for name in files:
+        path = os.path.join(ROOT, "head_latent_attention_05_b200", "csrc", name)
+        with open(path, encoding="utf-8") as f:
+            lines = [re.sub(r"//.*", "", ln).rstrip() for ln in f]
+        code += "\n".join(ln for ln in lines if ln.strip())
     return hashlib.sha256(code.encode()).hexdigest()[:16]
 
 

@@ -19,6 +19,8 @@ LIB_PATH = os.path.join(_HERE, "libmla.so")
 
 MLA_DTYPE_F32 = 0
 MLA_DTYPE_BF16 = 1
+MLA_KV_PLAIN = 0
+MLA_KV_FP8_E4M3 = 1
 
 STATUS = {
     0: "MLA_OK", 1: "MLA_ERR_INVALID_ARG", 2: "MLA_ERR_UNSUPPORTED",
@@ -33,7 +35,7 @@ EXPORTED = (
     "mla_prefill_ref_workspace_size",
     "mla_prefill_ref", "mla_get_device_error", "mla_query_workspace_size", "mla_query",
     "mla_output_workspace_size", "mla_output", "mla_decode_partial", "mla_combine_workspace_size",
-    "mla_combine", "mla_prefill_workspace_size", "mla_prefill",
+    "mla_combine", "mla_prefill_workspace_size", "mla_prefill", "mla_quantize_latent",
 )
 
 
@@ -50,17 +52,35 @@ class MlaConfig(ctypes.Structure):
         ("page_size", ctypes.c_int32), ("dtype", ctypes.c_int32),
         ("softmax_scale", ctypes.c_float), ("rms_eps", ctypes.c_float),
         ("rope_theta", ctypes.c_float), ("window", ctypes.c_int32),
+        ("kv_format", ctypes.c_int32),
     ]
 
 
 def make_config(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size=64, dtype="bf16",
-                softmax_scale=None, rms_eps=1e-6, rope_theta=10000.0, window=0) -> MlaConfig:
+                softmax_scale=None, rms_eps=1e-6, rope_theta=10000.0, window=0,
+                kv_format="plain") -> MlaConfig:
     if softmax_scale is None:
         softmax_scale = 1.0 / math.sqrt(d_nope + d_rope)
     dt = {"bf16": MLA_DTYPE_BF16, "f32": MLA_DTYPE_F32,
           torch.bfloat16: MLA_DTYPE_BF16, torch.float32: MLA_DTYPE_F32}[dtype]
+    kf = {"plain": MLA_KV_PLAIN, "fp8": MLA_KV_FP8_E4M3}[kv_format]
     return MlaConfig(n_heads, d_model, d_c, d_rope, d_nope, d_v, page_size, dt,
-                     softmax_scale, rms_eps, rope_theta, window)
+                     softmax_scale, rms_eps, rope_theta, window, kf)
+
+
+def fp8_page_bytes(cfg: MlaConfig) -> int:
+    """Bytes of one page of a quantised cache: page_size rows of d_c + d_rope codes, then the
+    page_size float32 scales (include/mla.h, mla_kv_format)."""
+    return cfg.page_size * (cfg.d_c + cfg.d_rope + 4)
+
+
+def fp8_cache_views(cfg: MlaConfig, cache: torch.Tensor):
+    """(codes [num_pages, page_size, d_c + d_rope] uint8, scales [num_pages, page_size] float32):
+    views of a quantised cache held as a uint8 tensor [num_pages, fp8_page_bytes(cfg)]."""
+    row, ps = cfg.d_c + cfg.d_rope, cfg.page_size
+    codes = cache[:, :ps * row].view(cache.shape[0], ps, row)
+    scales = cache[:, ps * row:].view(torch.float32)
+    return codes, scales
 
 
 _lib = None
@@ -110,6 +130,7 @@ def load_library() -> ctypes.CDLL:
         "mla_prefill_workspace_size": (SZ, [CFG, I32, I32]),
         "mla_prefill": (ctypes.c_int, [CFG, P, P, I32, I32, P, P, P, P, P, P, I32, P, I32, P, SZ,
                                        P, P]),
+        "mla_quantize_latent": (ctypes.c_int, [CFG, P, I32, P, P, P, I32, I32, P, I32, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -156,6 +177,14 @@ def mla_append_latent(cfg: MlaConfig, x, w_dkv, kv_gain, seq_idx, pos, block_tab
         _ptr(pos), _ptr(block_table), batch, max_pages, _ptr(cache), cache.shape[0],
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
         "mla_append_latent")
+
+
+def mla_quantize_latent(cfg: MlaConfig, rows, seq_idx, pos, block_table, cache, stream=None):
+    """Quantise float32 rows [n_tok, d_c + d_rope] into their slots of a quantised cache."""
+    batch, max_pages = block_table.shape
+    _check(load_library().mla_quantize_latent(
+        ctypes.byref(cfg), _ptr(rows), rows.shape[0], _ptr(seq_idx), _ptr(pos), _ptr(block_table),
+        batch, max_pages, _ptr(cache), cache.shape[0], _stream(stream)), "mla_quantize_latent")
 
 
 def mla_decode_workspace_size(cfg: MlaConfig, batch: int, tq: int) -> int:

@@ -18,6 +18,8 @@
 #include "ptx.cuh"
 #include "simt.cuh"
 #include "tc_decode.cuh"
+#include "tc_decode_fp8.cuh"
+#include "fp8_cache.cuh"
 #include "tc_gemm.cuh"
 #include "tc_vproj.cuh"
 
@@ -45,6 +47,7 @@ struct Carve {
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int elem_bytes(const mla_config* c) { return c->dtype == MLA_DTYPE_F32 ? 4 : 2; }
+bool fp8_cache(const mla_config* c) { return c->kv_format == MLA_KV_FP8_E4M3; }
 
 mla_status check_config(const mla_config* c) {
   if (c == nullptr) return MLA_ERR_INVALID_ARG;
@@ -55,9 +58,11 @@ mla_status check_config(const mla_config* c) {
   if (!(c->softmax_scale > 0.0f) || !std::isfinite(c->softmax_scale)) return MLA_ERR_INVALID_ARG;
   if (!(c->rms_eps >= 0.0f) || !(c->rope_theta > 0.0f)) return MLA_ERR_INVALID_ARG;
   if (c->window < 0) return MLA_ERR_INVALID_ARG;
-  // every row must stay 16-byte aligned for vector loads and TMA
-  const int64_t row_bytes = static_cast<int64_t>(c->d_c + c->d_rope) * elem_bytes(c);
+  if (c->kv_format != MLA_KV_PLAIN && c->kv_format != MLA_KV_FP8_E4M3) return MLA_ERR_INVALID_ARG;
+  // every row must stay 16-byte aligned for vector loads and TMA (a quantised row: its codes)
+  const int64_t row_bytes = static_cast<int64_t>(c->d_c + c->d_rope) * (fp8_cache(c) ? 1 : elem_bytes(c));
   if (row_bytes % 16 != 0) return MLA_ERR_UNSUPPORTED;
+  if (fp8_cache(c) && c->dtype != MLA_DTYPE_BF16) return MLA_ERR_UNSUPPORTED;
   if (c->d_rope > 2 * MLA_MAX_ROPE_PAIRS) return MLA_ERR_UNSUPPORTED;
   return MLA_OK;
 }
@@ -147,12 +152,13 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// Encoded maps are cached: a map is a pure function of (base, rank, dims, strides, box), so a
-// hit is always exact, and decode steps that reuse their buffers skip the driver call.
+// Encoded maps are cached: a map is a pure function of (base, rank, dims, strides, box, element
+// type, swizzle), so a hit is always exact, and decode steps that reuse their buffers skip the
+// driver call.
 struct MapKey {
-  uint64_t v[12];
+  uint64_t v[16];
   bool operator==(const MapKey& o) const {
-    for (int i = 0; i < 12; ++i)
+    for (int i = 0; i < 16; ++i)
       if (v[i] != o.v[i]) return false;
     return true;
   }
@@ -160,29 +166,48 @@ struct MapKey {
 struct MapKeyHash {
   size_t operator()(const MapKey& k) const {
     uint64_t h = 1469598103934665603ull;
-    for (int i = 0; i < 12; ++i) h = (h ^ k.v[i]) * 1099511628211ull;
+    for (int i = 0; i < 16; ++i) h = (h ^ k.v[i]) * 1099511628211ull;
     return static_cast<size_t>(h);
   }
 };
 constexpr size_t kMapCacheMax = 4096;
 
 bool encode_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                const uint64_t* strides_bytes, const uint32_t* box);
+                const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapDataType dt,
+                CUtensorMapSwizzle sw) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  cuuint64_t d[4], s[3];
+  cuuint32_t bx[4], es[4] = {1, 1, 1, 1};
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
+  return enc(m, dt, rank, const_cast<void*>(base), d, s, bx, es, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
-// bf16 tensor map with 128-byte swizzle. dims[0] is the contiguous dimension; strides are the
-// byte strides of dims 1.. ; box[0] must be 64 (one 128-byte swizzle row).
+// Tiled tensor map (rank <= 4). dims[0] is the contiguous dimension; strides are the byte
+// strides of dims 1.. . The default is bf16 with 128-byte swizzle (box[0] = 64 elements, one
+// swizzle row).
 bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-              const uint64_t* strides_bytes, const uint32_t* box) {
+              const uint64_t* strides_bytes, const uint32_t* box,
+              CUtensorMapDataType dt = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+              CUtensorMapSwizzle sw = CU_TENSOR_MAP_SWIZZLE_128B) {
   static std::mutex mu;
   static std::unordered_map<MapKey, CUtensorMap, MapKeyHash> cache;
+  if (rank < 1 || rank > 4) return false;
   MapKey k{};
   k.v[0] = reinterpret_cast<uint64_t>(base);
   k.v[1] = static_cast<uint64_t>(rank);
-  for (int i = 0; i < rank && i < 3; ++i) {
+  for (int i = 0; i < rank; ++i) {
     k.v[2 + i] = dims[i];
-    k.v[5 + i] = box[i];
+    k.v[6 + i] = box[i];
   }
-  for (int i = 0; i + 1 < rank && i < 2; ++i) k.v[8 + i] = strides_bytes[i];
+  for (int i = 0; i + 1 < rank; ++i) k.v[10 + i] = strides_bytes[i];
+  k.v[13] = static_cast<uint64_t>(dt);
+  k.v[14] = static_cast<uint64_t>(sw);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(k);
@@ -191,27 +216,11 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
       return true;
     }
   }
-  if (!encode_map(m, base, rank, dims, strides_bytes, box)) return false;
+  if (!encode_map(m, base, rank, dims, strides_bytes, box, dt, sw)) return false;
   std::lock_guard<std::mutex> lock(mu);
   if (cache.size() >= kMapCacheMax) cache.clear();
   cache.emplace(k, *m);
   return true;
-}
-
-bool encode_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims,
-                const uint64_t* strides_bytes, const uint32_t* box) {
-  EncodeTiledFn enc = encode_fn();
-  if (enc == nullptr) return false;
-  cuuint64_t d[3], s[2];
-  cuuint32_t bx[3], es[3] = {1, 1, 1};
-  for (int i = 0; i < rank; ++i) {
-    d[i] = dims[i];
-    bx[i] = box[i];
-  }
-  for (int i = 0; i + 1 < rank; ++i) s[i] = strides_bytes[i];
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), d, s, bx, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 // Raise a kernel's dynamic shared-memory limit, once per (kernel, device): later calls, which
@@ -663,6 +672,15 @@ mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok
   if (s != MLA_OK) return s;
   // the finish runs as clusters of FIN_CLUSTER CTAs per token (see append_finish_cluster_kernel)
   const int per = (((row + FIN_CLUSTER - 1) / FIN_CLUSTER) + 1) & ~1;
+  if (fp8_cache(cfg))
+    return launch_pdl_clustered(append_finish_cluster_fp8_kernel<FIN_CLUSTER>,
+                                dim3(static_cast<unsigned>(n_tok) * FIN_CLUSTER), dim3(FIN_THREADS),
+                                per * sizeof(float), st, FIN_CLUSTER,
+                                static_cast<const float*>(partial), ap.k_splits, n_tok,
+                                static_cast<const __nv_bfloat16*>(kv_gain), seq_idx, pos,
+                                block_table, batch, max_pages, static_cast<uint8_t*>(cache),
+                                num_pages, cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps,
+                                rope_freqs(cfg));
   return launch_pdl_clustered(append_finish_cluster_kernel<__nv_bfloat16>,
                               dim3(static_cast<unsigned>(n_tok) * FIN_CLUSTER), dim3(FIN_THREADS),
                               per * sizeof(float), st, FIN_CLUSTER,
@@ -671,6 +689,25 @@ mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok
                               block_table, batch, max_pages, static_cast<__nv_bfloat16*>(cache),
                               num_pages, cfg->page_size, cfg->d_c, cfg->d_rope, cfg->rms_eps,
                               rope_freqs(cfg));
+}
+
+mla_status mla_quantize_latent(const mla_config* cfg, const float* rows, int32_t n_tok,
+                               const int32_t* seq_idx, const int32_t* pos,
+                               const int32_t* block_table, int32_t batch, int32_t max_pages,
+                               void* cache, int32_t num_pages, void* stream) {
+  const mla_status cs = check_config(cfg);
+  if (cs != MLA_OK) return cs;
+  if (!fp8_cache(cfg)) return MLA_ERR_INVALID_ARG;
+  if (n_tok < 1 || batch < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
+  const void* ptrs[] = {rows, seq_idx, pos, block_table, cache};
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return MLA_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  quantize_rows_kernel<<<n_tok, 128, 0, st>>>(rows, n_tok, cfg->d_c + cfg->d_rope, seq_idx, pos,
+                                              block_table, batch, max_pages,
+                                              static_cast<uint8_t*>(cache), num_pages,
+                                              cfg->page_size);
+  return last_launch_status();
 }
 
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq) {
@@ -763,7 +800,30 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
   }
 
   // (2) fused latent attention, one partial per segment
-  {
+  if (fp8_cache(cfg)) {
+    // codes as [page][chunk of 128][token][128 codes] (two chunks per box) and the k_R codes as
+    // [page][token][64 codes] starting 512 bytes into the page; the scales follow the codes
+    CUtensorMap mc8, mr8;
+    const uint64_t dc[4] = {128, ATT_PAGE, ATT_DC / 128, static_cast<uint64_t>(num_pages)};
+    const uint64_t sc[3] = {ATT_ROW, 128, F8_PAGE_BYTES};
+    const uint32_t bc[4] = {128, ATT_PAGE, 2, 1};
+    const uint64_t dr[3] = {ATT_DR, ATT_PAGE, static_cast<uint64_t>(num_pages)};
+    const uint64_t sr[2] = {ATT_ROW, F8_PAGE_BYTES};
+    const uint32_t br[3] = {ATT_DR, ATT_PAGE, 1};
+    const uint8_t* c8 = static_cast<const uint8_t*>(cache);
+    if (!make_map(&mc8, c8, 4, dc, sc, bc, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mr8, c8 + ATT_DC, 3, dr, sr, br, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  CU_TENSOR_MAP_SWIZZLE_64B))
+      return MLA_ERR_CUDA;
+    AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
+                  max_pages, num_pages, H, tq, L.R, L.n_mt,
+                  cfg->softmax_scale * 1.4426950408889634f, keys, c8};
+    if (!allow_smem(mla_decode_attn_fp8_kernel, F8_SMEM_BYTES)) return MLA_ERR_CUDA;
+    mark(1);
+    const mla_status s = launch_pdl(mla_decode_attn_fp8_kernel, dim3(2 * L.P), dim3(F8_THREADS),
+                                    F8_SMEM_BYTES, st, mc8, mr8, ap);
+    if (s != MLA_OK) return s;
+  } else {
     CUtensorMap mc, mc4, mq;
     const uint64_t dc[2] = {ATT_ROW, static_cast<uint64_t>(num_pages) * ATT_PAGE};
     const uint64_t sc[1] = {ATT_ROW * 2};
@@ -779,7 +839,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
       return MLA_ERR_CUDA;
     AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
-                  cfg->softmax_scale * 1.4426950408889634f, keys};
+                  cfg->softmax_scale * 1.4426950408889634f, keys, nullptr};
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
     mark(1);
     const mla_status s = launch_pdl(mla_decode_attn_kernel, dim3(2 * L.P), dim3(ATT_THREADS),
@@ -1018,6 +1078,7 @@ mla_status mla_prefill(const mla_config* cfg, const void* x, const void* q, int3
                        size_t ws_bytes, void* out, void* stream) {
   const mla_status cs = check_config(cfg);
   if (cs != MLA_OK) return cs;
+  if (!tc_prefill_shape(cfg) && fp8_cache(cfg)) return MLA_ERR_UNSUPPORTED;
   if (!tc_prefill_shape(cfg))
     return mla_prefill_ref(cfg, x, q, batch, t_new, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens,
                            block_table, max_pages, cache, num_pages, workspace, ws_bytes, out,
@@ -1058,6 +1119,7 @@ mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, 
                            void* stream) {
   const mla_status cs = check_config(cfg);
   if (cs != MLA_OK) return cs;
+  if (fp8_cache(cfg)) return MLA_ERR_UNSUPPORTED;
   if (batch < 1 || t_new < 1 || max_pages < 1 || num_pages < 1) return MLA_ERR_INVALID_ARG;
   const void* ptrs[] = {x, q, w_dkv, kv_gain, w_uk_t, w_uv, seq_lens, block_table, cache,
                         workspace, out};

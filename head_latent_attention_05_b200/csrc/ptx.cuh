@@ -148,6 +148,26 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, u
       : "memory");
 }
 
+__device__ __forceinline__ void tma_load_4d(void* dst, const CUtensorMap* map, uint64_t* bar,
+                                            int32_t x, int32_t y, int32_t z, int32_t w) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6}], [%2];" ::"r"(smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_addr(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
+      : "memory");
+}
+
+// Plain (untiled) bulk copy global -> shared memory, completing on an mbarrier. Both addresses
+// 16-byte aligned, size a multiple of 16 bytes.
+__device__ __forceinline__ void bulk_load_g2s(void* dst, const void* src, uint32_t bytes,
+                                              uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_addr(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
 // Bring a contiguous global range into L2 ahead of use (no shared memory, no completion).
 // Address and size must be multiples of 16 bytes.
 __device__ __forceinline__ void prefetch_l2_bulk(const void* src, uint32_t bytes) {
@@ -269,6 +289,63 @@ __device__ __forceinline__ void mma_bf16_ss_x4_elect(uint32_t d_tmem, uint64_t a
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first)
       : "memory");
 }
+// The kind::f8f6f4 forms of the two chunk helpers above (E4M3 x E4M3 -> fp32): one 128-wide
+// K chunk of 8-bit operands is four K = 32 steps, and in the 128-byte swizzle and in TMEM a
+// K = 32 step of 8-bit elements covers the same 32 bytes / 8 columns as a K = 16 step of bf16,
+// so the operand addresses step exactly as in the bf16 forms.
+__device__ __forceinline__ void mma_f8_ts_x4_elect(uint32_t d_tmem, uint32_t a_tmem,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, t, e;\n\t.reg .b64 b1, b2, b3;\n\t.reg .b32 a1, a2, a3;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+      "add.u32 a1, %1, 8;\n\tadd.u32 a2, %1, 16;\n\tadd.u32 a3, %1, 24;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a1], b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a2], b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [a3], b3, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(acc_first)
+      : "memory");
+}
+__device__ __forceinline__ void mma_f8_ss_x4_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                   uint64_t b_desc, uint32_t idesc,
+                                                   uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, t, e;\n\t.reg .b64 a1, a2, a3, b1, b2, b3;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.s64 b1, %2, 2;\n\tadd.s64 b2, %2, 4;\n\tadd.s64 b3, %2, 6;\n\t"
+      "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a1, b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a2, b2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a3, b3, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(acc_first)
+      : "memory");
+}
+// Four accumulating K = 32 steps whose A operand walks a whole 128-byte row (descriptor
+// a_desc + 2*kk) while B repeats its first two steps (b_desc, b_desc + 2, b_desc, b_desc + 2):
+// A rows holding two 64-wide operands side by side (the high and low parts of a split value)
+// both meet the same 64-wide B.
+__device__ __forceinline__ void mma_f8_ss_pair_elect(uint32_t d_tmem, uint64_t a_desc,
+                                                     uint64_t b_desc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred t, e;\n\t.reg .b64 a1, a2, a3, b1;\n\t"
+      "setp.eq.b32 t, 0, 0;\n\t"
+      "add.s64 b1, %2, 2;\n\t"
+      "add.s64 a1, %1, 2;\n\tadd.s64 a2, %1, 4;\n\tadd.s64 a3, %1, 6;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a1, b1, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a2, %2, %3, t;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], a3, b1, %3, t;\n\t}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc)
+      : "memory");
+}
 __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -356,6 +433,27 @@ __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo
   d |= static_cast<uint64_t>(1) << 46;  // descriptor version for tcgen05
   d |= static_cast<uint64_t>(2) << 61;  // SWIZZLE_128B
   return d;
+}
+
+// The same with 64-byte swizzle (a TMA load with CU_TENSOR_MAP_SWIZZLE_64B and a 64-byte inner
+// box): K-major rows of 64 B, the pattern repeats every 8 rows x 64 B = 512 B (sbo).
+__device__ __forceinline__ uint64_t smem_desc_sw64(uint32_t saddr, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
+  d |= static_cast<uint64_t>(1) << 16;  // leading byte offset: unused for swizzled K-major
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;  // descriptor version for tcgen05
+  d |= static_cast<uint64_t>(4) << 61;  // SWIZZLE_64B
+  return d;
+}
+
+// Instruction descriptor, kind::f8f6f4 with E4M3 A/B (format code 0) and fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
+  return (1u << 4)                                    // D format: f32
+         | (0u << 7)                                  // A format: E4M3
+         | (0u << 10)                                 // B format: E4M3
+         | (static_cast<uint32_t>(N >> 3) << 17)      // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24);     // M / 16
 }
 
 // Instruction descriptor, kind::f16 with bf16 A/B and fp32 D.

@@ -88,6 +88,7 @@ struct AttnParams {
   int H, Tq, R, n_mt;
   float scale_log2;          // softmax_scale * log2(e)
   KeyRange keys;             // keys each query row may see (causal, window, key range)
+  const uint8_t* cache8;     // the quantised cache (fp8 kernel only: its pages' scales)
 };
 
 // ------------------------------------------------------------------------ split-KV planner
@@ -290,7 +291,8 @@ constexpr int ATT_SMEM_BYTES = ATT_STAGES * ATT_TILE_BYTES + ATT_QS_CHUNKS * ATT
                                static_cast<int>(sizeof(AttnShared));
 static_assert(ATT_SMEM_BYTES <= 227 * 1024, "attention kernel exceeds the shared memory of a CTA");
 
-__device__ __forceinline__ bool att_wait(AttnShared& sh, uint64_t* bar, uint32_t parity) {
+template <class SH>
+__device__ __forceinline__ bool att_wait(SH& sh, uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   while (true) {
@@ -306,7 +308,8 @@ __device__ __forceinline__ bool att_wait(AttnShared& sh, uint64_t* bar, uint32_t
 
 // Warp-uniform wait for the softmax warps (their TMEM loads/stores are warp-collective): lane 0
 // waits, the verdict is broadcast, then every lane acquires the completed phase itself.
-__device__ __forceinline__ bool att_warp_wait(AttnShared& sh, uint64_t* bar, uint32_t parity) {
+template <class SH>
+__device__ __forceinline__ bool att_warp_wait(SH& sh, uint64_t* bar, uint32_t parity) {
   bool ok = false;
   if ((threadIdx.x & 31) == 0) ok = att_wait(sh, bar, parity);
   ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;

@@ -60,6 +60,24 @@ typedef enum {
 typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1 } mla_dtype;
 
 /*
+ * How the latent cache stores a row (mla_config.kv_format).
+ * MLA_KV_PLAIN: rows of d_c + d_rope values in cfg->dtype; a page is
+ *   [page_size][d_c + d_rope] elements.
+ * MLA_KV_FP8_E4M3: the per-token quantised latent of
+ *   「Multi-Head Latent Attention（MLA）原理与工程实践全解析」 (one scale per token's whole latent
+ *   row). Each row is d_c + d_rope FP8 E4M3 codes (OCP E4M3: bias 7, largest finite 448, 0x7F /
+ *   0xFF are NaN) plus one float32 scale, and means code * scale. A page is
+ *   page_size * (d_c + d_rope + 4) bytes: the page_size rows of codes, token after token, then
+ *   the page_size scales. Quantising a row v (float32): scale = max|v| / 448, code_i =
+ *   E4M3(v_i / scale) (each a correctly rounded float32 division, then round to nearest, ties
+ *   to even, saturating at ±448); a row of zeros gets scale 0. It halves the cache's bytes; the
+ *   model's other tensors stay in cfg->dtype, which must be bf16. Decode, prefill and partial
+ *   decode run it on the tcgen05 path (its DeepSeek-V2 latent shapes); mla_prefill_ref and the
+ *   fp32 path do not take it (MLA_ERR_UNSUPPORTED).
+ */
+typedef enum { MLA_KV_PLAIN = 0, MLA_KV_FP8_E4M3 = 1 } mla_kv_format;
+
+/*
  * Model dimensions, named as in the page's module (「从零复现 DeepSeek-V2/V3 多头潜在注意力 MLA」
  * §2): n_heads, dim (d_model), kv_lora_rank (d_c), qk_rope_head_dim (d_rope),
  * qk_nope_head_dim (d_nope), v_head_dim (d_v). softmax_scale is normally
@@ -72,8 +90,9 @@ typedef enum { MLA_DTYPE_F32 = 0, MLA_DTYPE_BF16 = 1 } mla_dtype;
  * last 1024 latents, in 「Multi-Head Latent Attention（MLA）原理与工程实践全解析」 §7); 0 means
  * every earlier key (plain causal attention). The window applies to every decode and prefill
  * entry point; appends are unaffected.
- * Every entry point rejects d_rope > 128 with MLA_ERR_UNSUPPORTED, window < 0 with
- * MLA_ERR_INVALID_ARG.
+ * kv_format selects the cache's row format (mla_kv_format above).
+ * Every entry point rejects d_rope > 128 with MLA_ERR_UNSUPPORTED, window < 0 and an unknown
+ * kv_format with MLA_ERR_INVALID_ARG.
  */
 typedef struct {
   int32_t n_heads;
@@ -87,7 +106,8 @@ typedef struct {
   float softmax_scale;
   float rms_eps;
   float rope_theta;
-  int32_t window; /* 0 = unlimited */
+  int32_t window;    /* 0 = unlimited */
+  int32_t kv_format; /* mla_kv_format; 0 = rows in cfg->dtype */
 } mla_config;
 
 /* Human-readable name of a status code (static string). */
@@ -117,7 +137,8 @@ size_t mla_append_workspace_size(const mla_config* cfg, int32_t n_tok);
  *     c    = kv[:d_c] / sqrt(mean(kv[:d_c]^2) + rms_eps) * kv_gain
  *     k_R  = RoPE(kv[d_c:], pos[i])
  *     cache[block_table[seq_idx[i]][pos[i] / page_size]][pos[i] % page_size] = [c | k_R]
- * rounded once to cfg->dtype. fp32 accumulation.
+ * rounded once to cfg->dtype (with kv_format MLA_KV_FP8_E4M3: quantised from the float32 row,
+ * codes and scale; bf16 and d_model a multiple of 64 only). fp32 accumulation.
  *   x           [n_tok, d_model]
  *   w_dkv       [d_c + d_rope, d_model]     (wkv_a weight; rows [0,d_c) give c_KV)
  *   kv_gain     [d_c]                       (kv_norm weight)
@@ -125,6 +146,7 @@ size_t mla_append_workspace_size(const mla_config* cfg, int32_t n_tok);
  *   pos         [n_tok] int32, 0-based position in its sequence, < max_pages*page_size
  *   block_table [batch, max_pages] int32    page ids in [0, num_pages)
  *   cache       [num_pages, page_size, d_c + d_rope]   updated in place, only the addressed rows
+ *               (quantised: pages of page_size * (d_c + d_rope + 4) bytes, see mla_kv_format)
  *   workspace   >= mla_append_workspace_size(cfg, n_tok) bytes, 256-byte aligned
  * Tokens whose sequence, position or page is out of range are skipped and flagged
  * MLA_ERR_DEVICE_OOB. Two tokens addressing the same row race (caller's responsibility).
@@ -134,6 +156,22 @@ mla_status mla_append_latent(const mla_config* cfg, const void* x, int32_t n_tok
                              const int32_t* pos, const int32_t* block_table, int32_t batch,
                              int32_t max_pages, void* cache, int32_t num_pages, void* workspace,
                              size_t ws_bytes, void* stream);
+
+/*
+ * Write n_tok given rows into a quantised cache (kv_format MLA_KV_FP8_E4M3): row i is quantised
+ * as described at mla_kv_format and stored at position pos[i] of sequence seq_idx[i]. For
+ * filling such a cache from rows computed elsewhere (a bf16 cache being converted, rows from
+ * another model run); mla_append_latent computes and quantises new rows itself.
+ *   rows        [n_tok, d_c + d_rope] float32
+ *   seq_idx, pos, block_table, batch, max_pages, num_pages: as in mla_append_latent
+ *   cache       [num_pages] pages of page_size * (d_c + d_rope + 4) bytes, updated in place
+ * Tokens whose sequence, position or page is out of range are skipped and flagged
+ * MLA_ERR_DEVICE_OOB. Any kv_format other than MLA_KV_FP8_E4M3 is MLA_ERR_INVALID_ARG.
+ */
+mla_status mla_quantize_latent(const mla_config* cfg, const float* rows, int32_t n_tok,
+                               const int32_t* seq_idx, const int32_t* pos,
+                               const int32_t* block_table, int32_t batch, int32_t max_pages,
+                               void* cache, int32_t num_pages, void* stream);
 
 /* Bytes of workspace mla_decode needs for (batch, tq) on the current device (0 if invalid). */
 size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t tq);
@@ -147,7 +185,7 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t t
  * tokens 0 .. seq_lens[b] - tq + t (causal among the new tokens; a query sees itself —
  * 「淺析DeepSeek多頭潛在注意力機制（MLA）」: the new token attends to all N+1 keys).
  *   q           [batch, tq, n_heads, d_nope + d_rope]  un-rotated queries ([q_nope | q_rope])
- *   cache       [num_pages, page_size, d_c + d_rope]
+ *   cache       [num_pages, page_size, d_c + d_rope] (quantised: see mla_kv_format)
  *   block_table [batch, max_pages] int32
  *   seq_lens    [batch] int32 (device), each in [tq, max_pages*page_size]
  *   w_uk_t      [n_heads, d_c, d_nope], w_uv [n_heads, d_v, d_c]   (from mla_absorb_weights)

@@ -32,7 +32,14 @@ def assert_parity(got, ref, dtype: str, what: str = ""):
 
 def config_of(w: W.Workload) -> mla.MlaConfig:
     return mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, W.PAGE_SIZE, w.dtype,
-                           w.scale, w.rms_eps, w.rope_theta)
+                           w.scale, w.rms_eps, w.rope_theta, kv_format=w.kv)
+
+
+def fp8_views(w: W.Workload, cache: torch.Tensor):
+    """(codes [pages, 64, row] uint8, scales [pages, 64] float32) views of a quantised pool."""
+    n = W.PAGE_SIZE * w.row
+    return (cache[:, :n].view(cache.shape[0], W.PAGE_SIZE, w.row),
+            cache[:, n:].view(torch.float32))
 
 
 @dataclasses.dataclass
@@ -56,10 +63,18 @@ def make_case(w: W.Workload, lens: torch.Tensor | None = None, tail_fill=None,
     lens = W.seq_lens(w) if lens is None else lens.to(torch.int32)
     pt = W.page_table(w, lens)
     weights = W.weights(w)
-    cache = W.cache_pool(w, pt.num_pages)
-    if tail_fill is not None:
-        for page, slot in W.tail_slots(lens, pt):
-            cache[page, slot:] = tail_fill
+    if w.kv == "fp8":
+        cache = W.cache_pool_fp8(w, pt.num_pages)
+        if tail_fill is not None:   # stale slots: NaN codes and NaN scales
+            codes, scales = fp8_views(w, cache)
+            for page, slot in W.tail_slots(lens, pt):
+                codes[page, slot:] = 0x7F
+                scales[page, slot:] = float("nan")
+    else:
+        cache = W.cache_pool(w, pt.num_pages)
+        if tail_fill is not None:
+            for page, slot in W.tail_slots(lens, pt):
+                cache[page, slot:] = tail_fill
     x_new, seq_idx, pos, q = W.new_token_inputs(w, lens)
     cfg = config_of(w)
     cfg.window = window
@@ -103,8 +118,16 @@ def oracle_rows_of(c: Case, b: int, new_rows: np.ndarray) -> np.ndarray:
     rows for the last Tq positions."""
     w = c.w
     L = int(c.lens[b])
+    mine = new_rows[b * w.Tq:(b + 1) * w.Tq]
+    if w.kv == "fp8":
+        codes, scales = fp8_views(w, c.cache_host)
+        rows = O.gather_rows_fp8(codes.numpy(), scales.numpy(), c.pt.block_table[b].numpy(), L,
+                                 W.PAGE_SIZE)
+        qc, qs = O.quantize_rows_e4m3(mine.astype(np.float32))   # the oracle's own stored rows
+        rows[L - w.Tq:] = O.dequantize_rows_e4m3(qc, qs)
+        return rows
     rows = O.gather_rows(c.cache_host, c.pt.block_table[b].numpy(), L, W.PAGE_SIZE)
-    rows[L - w.Tq:] = new_rows[b * w.Tq:(b + 1) * w.Tq]
+    rows[L - w.Tq:] = mine
     return rows
 
 
@@ -139,9 +162,16 @@ def plant_score_staircase(c: Case, b: int, h: int, t: int = 0, base: float = 8.0
         row = np.zeros(w.row)
         row[:w.d_c] = (s / w.scale) * q_lat / float(q_lat @ q_lat)
         page = int(c.pt.block_table[b, page_i])
-        val = torch.from_numpy(row).to(w.torch_dtype)
-        c.cache_host[page, slot] = val
-        c.d["cache"][page, slot] = val.to(c.d["cache"].device)
+        if w.kv == "fp8":
+            qc, qs = O.quantize_rows_e4m3(row[None].astype(np.float32))
+            for cache in (c.cache_host, c.d["cache"]):
+                codes, scales = fp8_views(w, cache)
+                codes[page, slot] = torch.from_numpy(qc[0]).to(cache.device)
+                scales[page, slot] = float(qs[0])
+        else:
+            val = torch.from_numpy(row).to(w.torch_dtype)
+            c.cache_host[page, slot] = val
+            c.d["cache"][page, slot] = val.to(c.d["cache"].device)
         planted.append(j)
     return planted
 

@@ -101,3 +101,26 @@ def test_workspace_sizes_are_consistent(lib):
     assert mla.mla_decode_workspace_size(f32, 1, 1) >= (4 * (80 + 64)) * 4
     assert mla.mla_append_workspace_size(cfg, 16) >= 16 * 576 * 4
     assert mla.mla_prefill_ref_workspace_size(f32, 1, 128) > 0
+
+
+def test_quantised_cache_config_is_validated(lib):
+    fp8 = _cfg(kv_format="fp8")
+    assert _decode(lib, fp8, q=None) == 1                       # still validates pointers
+    assert _decode(lib, fp8, ws_bytes=16) == 3
+    bad = _cfg()
+    bad.kv_format = 2                                           # unknown row format
+    assert _decode(lib, bad) == 1
+    f32_fp8 = mla.make_config(4, 128, 64, 16, 32, 32, dtype="f32", kv_format="fp8")
+    assert _decode(lib, f32_fp8) == 2                           # quantised cache needs bf16
+    assert mla.mla_decode_workspace_size(fp8, 16, 1) == mla.mla_decode_workspace_size(_cfg(), 16, 1)
+    # mla_quantize_latent: only for a quantised cache, pointers checked before any launch
+    q = lambda cfg, rows=FAKE, n=4: lib.mla_quantize_latent(ctypes.byref(cfg), rows, n, FAKE, FAKE,
+                                                              FAKE, 2, 4, FAKE, 8, None)
+    assert q(_cfg()) == 1
+    assert q(fp8, rows=None) == 1
+    assert q(fp8, rows=ODD) == 1
+    assert q(fp8, n=0) == 1
+    # prefill_ref does not take a quantised cache
+    assert lib.mla_prefill_ref(ctypes.byref(fp8), FAKE, FAKE, 1, 1, FAKE, FAKE, FAKE, FAKE, FAKE,
+                               FAKE, 1, FAKE, 1, FAKE, 1 << 30, FAKE, None) == 2
+    assert mla.fp8_page_bytes(fp8) == 64 * (576 + 4)

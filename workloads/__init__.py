@@ -11,6 +11,11 @@ Distributions (chosen to match what the module on the pages produces with random
                                                     RoPE rotation of N(0,1) is again N(0,1)
   * q = [q_nope | q_rope] ~ N(0, 1)                -- RMSNorm'd q_a times a 1/fan_in weight
 The cache pool is filled i.i.d. page by page, so a shuffled page order is just a relabelling.
+
+A quantised cache (kv = "fp8": E4M3 codes plus one float32 scale per token, the page layout of
+include/mla.h) is drawn the same way: codes are N(0,1) draws times 448/4.5 cast to float8_e4m3fn
+by torch (so a row's codes reach about ±448, as a row quantised to its own maximum does), and
+each token's scale is 4.5/448 times a uniform factor in [0.75, 1.25].
 """
 
 from __future__ import annotations
@@ -43,6 +48,7 @@ class Workload:
     seed: int
     rms_eps: float = 1e-6
     rope_theta: float = 10000.0
+    kv: str = "plain"      # cache rows: "plain" (in dtype) | "fp8" (E4M3 codes + token scales)
 
     @property
     def scale(self) -> float:
@@ -55,6 +61,11 @@ class Workload:
     @property
     def torch_dtype(self):
         return torch.float32 if self.dtype == "f32" else torch.bfloat16
+
+    @property
+    def fp8_page_bytes(self) -> int:
+        """Bytes of one quantised cache page: 64 rows of codes, then 64 float32 scales."""
+        return PAGE_SIZE * (self.row + 4)
 
 
 # The five workloads: a tiny fp32 case, DeepSeek-V2 shape at batch 16 x 4096, the 32-head
@@ -83,6 +94,19 @@ WORKLOADS = {
 }
 
 WORKLOAD_ORDER = list(WORKLOADS)
+
+# The serving mix again over a quantised (FP8 E4M3, per-token scale) latent cache.
+EXTRA_WORKLOADS = {
+    "v2_fp8_b64_ctx1kto32k_mix": Workload(
+        "v2_fp8_b64_ctx1kto32k_mix", B=64, H=128, d_model=5120, d_c=512, d_r=64,
+        d_nope=128, d_v=128, q_lora=1536, Tq=1, lens=("loguniform", 1024, 32768),
+        dtype="bf16", pages="shuffled", seed=3, kv="fp8"),
+}
+
+
+def get(name: str) -> Workload:
+    """A workload by name, from WORKLOADS or EXTRA_WORKLOADS."""
+    return WORKLOADS[name] if name in WORKLOADS else EXTRA_WORKLOADS[name]
 
 
 def small_variant(w: Workload, **over) -> Workload:
@@ -183,6 +207,21 @@ def cache_pool(w: Workload, num_pages: int, chunk_pages: int = 2048) -> torch.Te
     for i, p0 in enumerate(range(0, num_pages, chunk_pages)):
         p1 = min(num_pages, p0 + chunk_pages)
         out[p0:p1] = randn((p1 - p0, PAGE_SIZE, w.row), w.seed, 1000 + i, 1.0, w.torch_dtype)
+    return out
+
+
+def cache_pool_fp8(w: Workload, num_pages: int, chunk_pages: int = 2048) -> torch.Tensor:
+    """Quantised page pool as bytes [num_pages, fp8_page_bytes]: per page 64 rows of E4M3 codes
+    (row after row), then the 64 float32 token scales (see the module docstring)."""
+    n_codes = PAGE_SIZE * w.row
+    out = torch.empty((num_pages, w.fp8_page_bytes), dtype=torch.uint8)
+    for i, p0 in enumerate(range(0, num_pages, chunk_pages)):
+        p1 = min(num_pages, p0 + chunk_pages)
+        v = randn((p1 - p0, n_codes), w.seed, 1000 + i, 448.0 / 4.5, torch.float32)
+        out[p0:p1, :n_codes] = v.clamp_(-448.0, 448.0).to(torch.float8_e4m3fn).view(torch.uint8)
+        u = torch.rand((p1 - p0, PAGE_SIZE), generator=_gen(w.seed, 3000 + i), dtype=torch.float32)
+        scales = (4.5 / 448.0) * (0.75 + 0.5 * u)
+        out[p0:p1, n_codes:] = scales.view(torch.uint8).view(p1 - p0, 4 * PAGE_SIZE)
     return out
 
 
