@@ -55,15 +55,6 @@ __device__ __forceinline__ uint16_t e4m3_encode2(float v0, float v1, float scale
   return static_cast<uint16_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(v0, v1), __NV_SATFINITE, __NV_E4M3));
 }
-// Two E4M3 codes (low byte first) as a bf16 pair, exactly (every E4M3 value is a bf16 value).
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t two) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  __half_raw lo, hi;
-  lo.x = h.x;
-  hi.x = h.y;
-  return pack_bf16x2(__half2float(__half(lo)), __half2float(__half(hi)));
-}
-
 // Quantise n_tok float32 rows [n_tok][row] into their cache slots: one block per token (even
 // row, blockDim a multiple of 32). Out-of-range tokens are skipped and flagged DEVICE_OOB.
 __global__ void __launch_bounds__(256)

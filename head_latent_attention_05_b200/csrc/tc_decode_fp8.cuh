@@ -72,13 +72,26 @@ __device__ __forceinline__ uint16_t e4m3x2_raw(float a, float b) {
   return static_cast<uint16_t>(
       __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3));
 }
-__device__ __forceinline__ void e4m3x2_to_f32(uint16_t two, float& a, float& b) {
-  const __half2_raw h = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(two), __NV_E4M3);
-  __half_raw lo, hi;
-  lo.x = h.x;
-  hi.x = h.y;
-  a = __half2float(__half(lo));
-  b = __half2float(__half(hi));
+// Value of an E4M3 code (low byte of c) in float32, exactly, without the conversion pipe: the
+// code's exponent and mantissa bits placed in a float32's exponent and mantissa fields make a
+// float32 equal to the value times 2^-120 (subnormal codes become float32 denormals, which
+// keep every bit), and the multiplication by 2^120 is exact.
+__device__ __forceinline__ float e4m3_value_f32(uint32_t c) {
+  return __uint_as_float(((c & 0x80u) << 24) | ((c & 0x7Fu) << 20)) * 0x1p120f;
+}
+// Four E4M3 codes (one 32-bit word, first code in the lowest byte) as two bf16 pairs, exactly,
+// in the same way: each code's bits placed in a bf16 lane give the value times 2^-120 (a bf16
+// denormal for a subnormal code), and one bf16x2 multiplication by 2^120 restores it.
+__device__ __forceinline__ void e4m3x4_to_bf16x4(uint32_t x, uint32_t& lo, uint32_t& hi) {
+  const __nv_bfloat162 k = __halves2bfloat162(__ushort_as_bfloat16(0x7B80), __ushort_as_bfloat16(0x7B80));
+  const uint32_t t0 = __byte_perm(x, 0u, 0x1404);   // lanes: code 0 << 8, code 1 << 8
+  const uint32_t t1 = __byte_perm(x, 0u, 0x3424);   // lanes: code 2 << 8, code 3 << 8
+  const uint32_t v0 = (t0 & 0x80008000u) | ((t0 >> 4) & 0x07F007F0u);
+  const uint32_t v1 = (t1 & 0x80008000u) | ((t1 >> 4) & 0x07F007F0u);
+  const __nv_bfloat162 r0 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v0), k);
+  const __nv_bfloat162 r1 = __hmul2(*reinterpret_cast<const __nv_bfloat162*>(&v1), k);
+  lo = *reinterpret_cast<const uint32_t*>(&r0);
+  hi = *reinterpret_cast<const uint32_t*>(&r1);
 }
 // Eight bf16 query values times inv -> their high and low E4M3 parts (two 32-bit words each,
 // the first feature in the lowest byte).
@@ -91,8 +104,7 @@ __device__ __forceinline__ void f8_split8(const uint4& x, float inv, uint32_t& h
     const float a = __uint_as_float(w[i] << 16) * inv;
     const float b = __uint_as_float(w[i] & 0xFFFF0000u) * inv;
     const uint16_t hh = e4m3x2_raw(a, b);
-    float ha, hb;
-    e4m3x2_to_f32(hh, ha, hb);
+    const float ha = e4m3_value_f32(hh), hb = e4m3_value_f32(static_cast<uint32_t>(hh) >> 8);
     hc[i] = hh;
     lc[i] = e4m3x2_raw(a - ha, b - hb);   // exact differences (ha, hb are a, b rounded)
   }
@@ -158,7 +170,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       mbar_init(&sh.full_qk[s], 1);
       mbar_init(&sh.full_own[s], 1);
       mbar_init(&sh.empty_qk[s], 1);
-      mbar_init(&sh.empty_own[s], 1);
+      mbar_init(&sh.empty_own[s], 1);   // committed after the stage's P·C
       mbar_init(&sh.cv_full[s], F8_CONV_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
@@ -331,6 +343,8 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           visible_keys(p.keys, b, L, p.Tq, (mt * 128) / p.H, &lo_u, &unused);
           visible_keys(p.keys, b, L, p.Tq, min(p.Tq - 1, (mt * 128 + 127) / p.H), &unused, &hi_u);
         }
+        // the own chunks of tile g land only after P·C of tile g-2, which read this stage's
+        // converted buffer
         if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
         const int z_lo = min(ATT_PAGE, max(0, lo_u - cur.tile * ATT_PAGE));
         const int z_keep = max(z_lo, min(ATT_PAGE, hi_u + 1 - cur.tile * ATT_PAGE));
@@ -344,14 +358,10 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
           if (r >= z_lo && r < z_keep) {
             const uint4 x = *reinterpret_cast<const uint4*>(src + j * F8_CHUNK_BYTES + r * 128 + ((u ^ sw) << 4));
-            lo4.x = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.x));
-            lo4.y = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.x >> 16));
-            lo4.z = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.y));
-            lo4.w = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.y >> 16));
-            hi4.x = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.z));
-            hi4.y = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.z >> 16));
-            hi4.z = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.w));
-            hi4.w = e4m3x2_to_bf16x2(static_cast<uint16_t>(x.w >> 16));
+            e4m3x4_to_bf16x4(x.x, lo4.x, lo4.y);
+            e4m3x4_to_bf16x4(x.y, lo4.z, lo4.w);
+            e4m3x4_to_bf16x4(x.z, hi4.x, hi4.y);
+            e4m3x4_to_bf16x4(x.w, hi4.z, hi4.w);
           }
           // features 16u .. 16u+15 of source chunk j: bf16 chunk 2j + u/4, 16-byte units
           // 2(u%4) and 2(u%4) + 1 of row r

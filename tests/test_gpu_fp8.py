@@ -277,3 +277,37 @@ def test_fp8_partials_merge_to_decode():
         Hs.assert_parity(got, o_ref, "bf16", f"fp8 partial b={b}")
         ref = Hs.oracle_out(c, b, [0, 64, 127], new_rows)
         Hs.assert_parity(out.float().cpu()[b][:, [0, 64, 127]], ref, "bf16", f"fp8 merged b={b}")
+
+
+def test_fp8_subnormal_codes_keep_their_values():
+    """History rows made only of subnormal codes (±m·2^-9, m = 1..7): decoding just those keys
+    (a key range that leaves out the appended token) must see their exact values, in the score
+    and in the value product; a conversion that flushed them would return zeros."""
+    w = W.small_variant(V2, B=2)
+    c = Hs.make_case(w, _lens(300, 129))
+    g = torch.Generator().manual_seed(5)
+    shape = (c.pt.num_pages, W.PAGE_SIZE, w.row)
+    sub = torch.randint(1, 8, shape, generator=g, dtype=torch.uint8)
+    sub |= torch.randint(0, 2, shape, generator=g, dtype=torch.uint8) << 7
+    for cache in (c.cache_host, c.d["cache"]):
+        codes, scales = Hs.fp8_views(w, cache)
+        codes.copy_(sub.to(cache.device))
+        scales.fill_(64.0)   # row values m/8: far above the parity bound's absolute term
+    Hs.run_append(c)
+    rows_n = w.B * w.Tq * w.H
+    o = torch.empty((rows_n, w.d_c), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty(rows_n, dtype=torch.float32, device="cuda")
+    ws = mla.workspace(mla.mla_decode_workspace_size(c.cfg, w.B, w.Tq))
+    kb = torch.zeros(w.B, dtype=torch.int32)
+    ke = c.lens - 1
+    mla.mla_decode_partial(c.cfg, c.d["q"], c.d["cache"], c.d["block_table"], c.d["seq_lens"],
+                           kb.cuda(), ke.cuda(), c.d["w_uk_t"], ws, o, lse)
+    got = o.float().cpu().view(w.B, w.Tq, w.H, w.d_c)
+    new_rows = Hs.oracle_new_rows(c)
+    W_UK, _ = O.split_wkv_b(c.weights.wkv_b, w.H, w.d_nope, w.d_v)
+    for b in range(w.B):
+        rows = Hs.oracle_rows_of(c, b, new_rows)
+        o_ref, _ = O.latent_partial(c.q[b], rows, W_UK, w.scale, w.rope_theta, 0, int(ke[b]),
+                                    heads=[0, 64, 127])
+        assert np.max(np.abs(o_ref)) > 0
+        Hs.assert_parity(got[b][:, [0, 64, 127]], o_ref, "bf16", f"subnormal codes b={b}")
