@@ -330,6 +330,8 @@ struct DecodeLayout {
   __nv_bfloat16* qhat;
   __nv_bfloat16* o_part;
   float* lse;
+  uint8_t* qcodes;   // quantised cache only: the split query rows and their scales
+  float* qalpha;
   size_t bytes;
 };
 
@@ -357,6 +359,10 @@ DecodeLayout decode_layout_tc(const mla_config* c, int B, int Tq, void* ws) {
   L.qhat = cv.take<__nv_bfloat16>(static_cast<size_t>(B) * L.R * ATT_ROW);
   L.o_part = cv.take<__nv_bfloat16>(static_cast<size_t>(L.max_segs) * 128 * ATT_DC);
   L.lse = cv.take<float>(static_cast<size_t>(L.max_segs) * 128);
+  if (fp8_cache(c)) {
+    L.qcodes = cv.take<uint8_t>(static_cast<size_t>(B) * L.R * F8_QROW_BYTES);
+    L.qalpha = cv.take<float>(static_cast<size_t>(B) * L.R);
+  }
   L.bytes = cv.off;
   return L;
 }
@@ -810,18 +816,30 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
     const uint64_t dr[3] = {ATT_DR, ATT_PAGE, static_cast<uint64_t>(num_pages)};
     const uint64_t sr[2] = {ATT_ROW, F8_PAGE_BYTES};
     const uint32_t br[3] = {ATT_DR, ATT_PAGE, 1};
+    // the split query rows: [row][1152 bytes], five 128-byte chunks per box row
+    CUtensorMap mq8;
+    const uint64_t dq[2] = {F8_QROW_BYTES, static_cast<uint64_t>(batch) * L.R};
+    const uint64_t sq[1] = {F8_QROW_BYTES};
+    const uint32_t bq[2] = {128, 128};
     const uint8_t* c8 = static_cast<const uint8_t*>(cache);
     if (!make_map(&mc8, c8, 4, dc, sc, bc, CU_TENSOR_MAP_DATA_TYPE_UINT8, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !make_map(&mr8, c8 + ATT_DC, 3, dr, sr, br, CU_TENSOR_MAP_DATA_TYPE_UINT8,
-                  CU_TENSOR_MAP_SWIZZLE_64B))
+                  CU_TENSOR_MAP_SWIZZLE_64B) ||
+        !make_map(&mq8, L.qcodes, 2, dq, sq, bq, CU_TENSOR_MAP_DATA_TYPE_UINT8,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
       return MLA_ERR_CUDA;
+    // Q̂ rows -> their high and low E4M3 parts and row scales
+    const int n_rows = batch * L.R;
+    mla_status s = launch_pdl(qsplit_rows_kernel, dim3((n_rows + 7) / 8), dim3(256), 0, st,
+                              static_cast<const __nv_bfloat16*>(L.qhat), n_rows, L.qcodes, L.qalpha);
+    if (s != MLA_OK) return s;
     AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
-                  cfg->softmax_scale * 1.4426950408889634f, keys, c8};
+                  cfg->softmax_scale * 1.4426950408889634f, keys, c8, L.qcodes, L.qalpha};
     if (!allow_smem(mla_decode_attn_fp8_kernel, F8_SMEM_BYTES)) return MLA_ERR_CUDA;
     mark(1);
-    const mla_status s = launch_pdl(mla_decode_attn_fp8_kernel, dim3(2 * L.P), dim3(F8_THREADS),
-                                    F8_SMEM_BYTES, st, mc8, mr8, ap);
+    s = launch_pdl(mla_decode_attn_fp8_kernel, dim3(2 * L.P), dim3(F8_THREADS), F8_SMEM_BYTES, st,
+                   mc8, mr8, mq8, ap);
     if (s != MLA_OK) return s;
   } else {
     CUtensorMap mc, mc4, mq;
@@ -839,7 +857,7 @@ static mla_status decode_impl(const mla_config* cfg, const void* q, int32_t batc
       return MLA_ERR_CUDA;
     AttnParams ap{block_table, seq_lens, L.segs, L.pair_seg, L.qhat, L.o_part, L.lse,
                   max_pages, num_pages, H, tq, L.R, L.n_mt,
-                  cfg->softmax_scale * 1.4426950408889634f, keys, nullptr};
+                  cfg->softmax_scale * 1.4426950408889634f, keys, nullptr, nullptr, nullptr};
     if (!allow_smem(mla_decode_attn_kernel, ATT_SMEM_BYTES)) return MLA_ERR_CUDA;
     mark(1);
     const mla_status s = launch_pdl(mla_decode_attn_kernel, dim3(2 * L.P), dim3(ATT_THREADS),

@@ -88,7 +88,9 @@ struct AttnParams {
   int H, Tq, R, n_mt;
   float scale_log2;          // softmax_scale * log2(e)
   KeyRange keys;             // keys each query row may see (causal, window, key range)
-  const uint8_t* cache8;     // the quantised cache (fp8 kernel only: its pages' scales)
+  const uint8_t* cache8;     // fp8 kernel only: the quantised cache (its pages' scales),
+  const uint8_t* qcodes;     //   the split query rows [B*R][1152] (qsplit_rows_kernel)
+  const float* qalpha;       //   and their scales [B*R]
 };
 
 // ------------------------------------------------------------------------ split-KV planner

@@ -11,7 +11,9 @@
 //     Q̂_r / a_r = hi_r + lo_r + (error of about 2^-8 relative),   hi = E4M3(Q̂_r / a_r),
 //                                                                lo = E4M3(Q̂_r / a_r - hi),
 // and both parts multiply the same codes: D_rj = (hi_r + lo_r) · K_j, two MMAs per K-step into
-// one accumulator. The softmax then works with s_rj = D_rj * sc_j * (a_r * scale). This costs
+// one accumulator. The softmax then works with s_rj = D_rj * sc_j * (a_r * scale). The split is
+// its own small kernel (qsplit_rows_kernel), run between the query absorption and this kernel,
+// which lays every row out as the attention kernel loads it (F8_QROW_BYTES below). This costs
 // the same tensor time as the bf16 kernel's score (twice the MMAs at twice the rate) and keeps
 // its precision (bf16 also keeps about 8 bits), while each page is half the bytes.
 //
@@ -27,8 +29,8 @@
 // the barriers. TMEM: [0,256) O half, [256,384) two score buffers, [384,448) hi and [448,512) lo
 // of the query's features 0..255 (four codes per column).
 //
-// Warp roles (448 threads): 0 TMA producer, 1 MMA issuer, 2..9 softmax (they also split and
-// place each unit's query), 10..13 converters.
+// Warp roles (448 threads): 0 TMA producer, 1 MMA issuer, 2..9 softmax (they also place each
+// unit's query features 0..255 in TMEM), 10..13 converters.
 #pragma once
 
 #include "fp8_cache.cuh"
@@ -54,11 +56,11 @@ struct AttnSharedF8 {
   uint64_t empty_qk[ATT_STAGES], empty_own[ATT_STAGES];
   uint64_t cv_full[ATT_STAGES];        // converters wrote the stage's bf16 c_KV half
   uint64_t s_full[2], p_full[2], pv_done[2];
-  uint64_t q_full;                     // the softmax warps placed a unit's split query
+  uint64_t q_full;                     // the softmax warps placed a unit's query in TMEM
+  uint64_t qs_full;                    // the unit's query chunks landed in shared memory (TMA)
   uint64_t q_free, o_free, drain;
   uint64_t pair_bar[4];
   float row_max[2][2][128];
-  float q_amax[2][128];                // each half row's largest |Q̂|
   uint32_t tmem_base;
   volatile int abort_flag;
 };
@@ -122,6 +124,53 @@ __device__ __forceinline__ float absmax_bf16x8(const uint4& x) {
   return m;
 }
 
+// A split query row, 1152 bytes: [hi 0..255 | lo 0..255 | hi 256..511 | lo 256..511 |
+// hi 512..575, lo 512..575] (feature indices; one code per feature). The first 512 bytes go to
+// TMEM, the other 640 are the five [128 rows x 128 B] shared-memory chunks of the kernel, each
+// one TMA box.
+constexpr int F8_QROW_BYTES = 2 * ATT_ROW;
+__device__ __forceinline__ int qsplit_hi_pos(int f) {
+  return f < 256 ? f : (f < 512 ? 512 + (f - 256) : 1024 + (f - 512));
+}
+__device__ __forceinline__ int qsplit_lo_pos(int f) {
+  return f < 256 ? 256 + f : (f < 512 ? 768 + (f - 256) : 1088 + (f - 512));
+}
+
+// Split n_rows bf16 query rows [n_rows][576] into their high and low E4M3 parts under the row's
+// scale a = max|row| / 448 (0 for a zero row): codes [n_rows][1152] in the layout above and
+// a [n_rows]. One warp per row, 8 rows per 256-thread block; lane l takes 8-feature groups l,
+// l + 32 and l + 64 (< 72).
+__global__ void __launch_bounds__(256)
+qsplit_rows_kernel(const __nv_bfloat16* __restrict__ qhat, int n_rows, uint8_t* __restrict__ codes,
+                   float* __restrict__ alpha) {
+  pdl_wait();   // the query absorption just before wrote qhat
+  pdl_trigger();
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5), lane = threadIdx.x & 31;
+  if (row >= n_rows) return;
+  const uint4* src = reinterpret_cast<const uint4*>(qhat + static_cast<int64_t>(row) * ATT_ROW);
+  uint4 x[3];
+  float am = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int gi = lane + 32 * k;
+    x[k] = gi < ATT_ROW / 8 ? src[gi] : make_uint4(0, 0, 0, 0);
+    am = fmaxf(am, absmax_bf16x8(x[k]));
+  }
+  am = warp_max(am);
+  const float inv = am > 0.0f ? __fdiv_rn(E4M3_MAX_F, am) : 0.0f;
+  uint8_t* dst = codes + static_cast<int64_t>(row) * F8_QROW_BYTES;
+#pragma unroll
+  for (int k = 0; k < 3; ++k) {
+    const int gi = lane + 32 * k;
+    if (gi >= ATT_ROW / 8) break;
+    uint2 h, l;
+    f8_split8(x[k], inv, h.x, h.y, l.x, l.y);
+    *reinterpret_cast<uint2*>(dst + qsplit_hi_pos(8 * gi)) = h;
+    *reinterpret_cast<uint2*>(dst + qsplit_lo_pos(8 * gi)) = l;
+  }
+  if (lane == 0) alpha[row] = __fdiv_rn(am, E4M3_MAX_F);
+}
+
 // Score K-steps of one 128-code chunk c of a page into the score buffer at TMEM column d_s:
 // the hi and the lo part of the query each meet the chunk's four K = 32 steps. Chunks 0, 1
 // take A from TMEM, chunks 2, 3 from shared memory (query chunks c-2 (hi) and c (lo)).
@@ -150,7 +199,8 @@ __device__ __forceinline__ void f8_qk_rope(uint32_t tmem, uint32_t d_s, uint32_t
 
 __global__ void __launch_bounds__(F8_THREADS, 1)
 mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
-                           const __grid_constant__ CUtensorMap map_r8, AttnParams p) {
+                           const __grid_constant__ CUtensorMap map_r8,
+                           const __grid_constant__ CUtensorMap map_q8, AttnParams p) {
   extern __shared__ __align__(1024) uint8_t smem[];
   if ((smem_addr(smem) & 1023u) != 0) {
     if (threadIdx.x == 0) record_error(MLA_ERR_UNSUPPORTED);
@@ -179,6 +229,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       mbar_init(&sh.pv_done[b], 1);
     }
     mbar_init(&sh.q_full, ATT_SM_WARPS);
+    mbar_init(&sh.qs_full, 1);
     mbar_init(&sh.q_free, 1);
     mbar_init(&sh.o_free, ATT_SM_WARPS);
     mbar_init(&sh.drain, 1);
@@ -187,6 +238,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
     fence_mbar_init();
     tma_prefetch_desc(&map_c8);
     tma_prefetch_desc(&map_r8);
+    tma_prefetch_desc(&map_q8);
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, 512);
@@ -232,20 +284,30 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
             tma_load_3d(st + 4 * F8_CHUNK_BYTES, &map_r8, bar, 0, 0, page);
           }
         };
+        int n_qloads = 0;   // query loads issued: the last one is drained before the CTA leaves
+        auto load_q_smem = [&](const AttnSeg& sg) {   // query bytes 512..1151 of a unit's rows
+          const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
+          mbar_arrive_expect_tx(&sh.qs_full, F8_QS_CHUNKS * F8_QS_CHUNK_BYTES);
+          for (int c = 0; c < F8_QS_CHUNKS; ++c)
+            tma_load_2d(qs_buf + c * F8_QS_CHUNK_BYTES, &map_q8, &sh.qs_full, 512 + 128 * c,
+                        b * p.R + mt * 128);
+          ++n_qloads;
+        };
         TileCursor cq, co;   // score-only cursor (one tile ahead), own-chunk cursor
         cq.init(p.segs, seg_begin, seg_end);
         co.init(p.segs, seg_begin, seg_end);
-        if (half == 0) {   // later segments' Q̂ rows into L2
+        if (half == 0) {   // later segments' query rows into L2
           for (int s_i = seg_begin + 1; s_i < seg_end; ++s_i) {
             const AttnSeg sg = p.segs[s_i];
             const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
             const int rows = min(128, p.R - mt * 128);
-            prefetch_l2_bulk(p.qhat + (static_cast<int64_t>(b) * p.R + mt * 128) * ATT_ROW,
-                             static_cast<uint32_t>(rows * ATT_ROW * 2));
+            prefetch_l2_bulk(p.qcodes + (static_cast<int64_t>(b) * p.R + mt * 128) * F8_QROW_BYTES,
+                             static_cast<uint32_t>(rows * F8_QROW_BYTES));
           }
         }
         int gq = 0, go = 0;
         bool ok = true;
+        load_q_smem(cq.sg);
         load_chunks(cq, gq, false, &sh.full_qk[0]);
         cq.next();
         ++gq;
@@ -256,9 +318,15 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
             break;
           }
           load_chunks(co, go, true, &sh.full_own[st]);
+          const bool seg_ends = co.last_of_seg();
+          const int k_done = co.k;
           co.next();
           ++go;
           if (!cq.valid()) continue;
+          if (seg_ends) {   // the next unit's query chunks: the last S of this one must be done
+            if (!att_wait(sh, &sh.q_free, k_done & 1)) { ok = false; break; }
+            load_q_smem(cq.sg);
+          }
           st = gq % ATT_STAGES;
           if (gq >= ATT_STAGES && !att_wait(sh, &sh.empty_qk[st], ((gq / ATT_STAGES) - 1) & 1)) {
             ok = false;
@@ -268,7 +336,9 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           cq.next();
           ++gq;
         }
-        // drain: the last loads of each ring must land before the CTA can exit
+        // drain: the last query load and the last loads of each ring must land before the CTA
+        // can exit
+        if (n_qloads > 0) (void)mbar_wait(&sh.qs_full, (n_qloads - 1) & 1);
         for (int j = max(0, gq - ATT_STAGES); j < gq; ++j)
           (void)mbar_wait(&sh.full_qk[j % ATT_STAGES], (j / ATT_STAGES) & 1);
         for (int j = max(0, go - ATT_STAGES); j < go; ++j)
@@ -298,7 +368,11 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       for (; cur.valid(); ++g, cur.next()) {
         const int st = g % ATT_STAGES, sb = g & 1;
         const uint32_t d_s = TM_S + 64 * sb;
-        if (cur.first_of_seg() && !att_warp_wait(sh, &sh.q_full, cur.k & 1)) { ok = false; break; }
+        if (cur.first_of_seg() && (!att_warp_wait(sh, &sh.q_full, cur.k & 1) ||
+                                   !att_warp_wait(sh, &sh.qs_full, cur.k & 1))) {
+          ok = false;
+          break;
+        }
         if (g >= 2 && !att_warp_wait(sh, &sh.pv_done[sb], ((g >> 1) - 1) & 1)) { ok = false; break; }
         const uint32_t st_addr = stage0 + st * F8_STAGE_BYTES;
         const uint64_t b_stage = smem_desc_sw128(st_addr, 16, 1024);
@@ -389,65 +463,27 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
         ++xc;
         return r;
       };
-      // A unit's query rows split into hi and lo E4M3 parts under the row's scale; features
-      // 0..255 into TMEM (warps of column half 0), 256..575 into the shared chunks (half 1).
-      // Returns false on abort; *rowf = a_r * softmax_scale * log2(e).
+      // A unit's split query features 0..255 into TMEM (row r_local; zeros past the unit):
+      // the warps of column half 0 write the hi codes, those of half 1 the lo codes. Returns
+      // false on abort; *rowf = a_r * softmax_scale * log2(e).
       auto load_q = [&](const AttnSeg& sg, float* rowf) -> bool {
         const int b = sg.unit / p.n_mt, mt = sg.unit % p.n_mt;
         const int r_in = mt * 128 + r_local;
         const bool valid = r_in < p.R;
-        const uint4* src = reinterpret_cast<const uint4*>(
-            p.qhat + (static_cast<int64_t>(b) * p.R + (valid ? r_in : 0)) * ATT_ROW);
-        const uint4 z4 = make_uint4(0, 0, 0, 0);
-        float am = 0.0f;
-        if (valid) {
-          const int k0 = hc ? 32 : 0, k1 = hc ? 72 : 32;
-#pragma unroll 8
-          for (int k = k0; k < k1; ++k) am = fmaxf(am, absmax_bf16x8(src[k]));
-        }
-        sh.q_amax[hc][r_local] = am;
-        if (!meet()) return false;
-        const float amax = fmaxf(sh.q_amax[0][r_local], sh.q_amax[1][r_local]);
-        const float inv = amax > 0.0f ? __fdiv_rn(E4M3_MAX_F, amax) : 0.0f;
-        *rowf = __fdiv_rn(amax, E4M3_MAX_F) * p.scale_log2;
-        if (hc == 0) {
+        const int64_t grow = static_cast<int64_t>(b) * p.R + (valid ? r_in : 0);
+        const uint4* src = reinterpret_cast<const uint4*>(p.qcodes + grow * F8_QROW_BYTES + 256 * hc);
+        *rowf = valid ? p.qalpha[grow] * p.scale_log2 : 0.0f;
+        uint32_t v[32];
 #pragma unroll 1
-          for (int j = 0; j < 4; ++j) {   // 64 features: 16 TMEM columns of hi and of lo
-            uint32_t hw[16], lw[16];
+        for (int c = 0; c < 2; ++c) {
 #pragma unroll
-            for (int u = 0; u < 8; ++u) {
-              const uint4 x = valid ? src[8 * j + u] : z4;
-              f8_split8(x, inv, hw[2 * u], hw[2 * u + 1], lw[2 * u], lw[2 * u + 1]);
-            }
-            tmem_st16(tmem + t_lane + TM_QHI + 16 * j, hw);
-            tmem_st16(tmem + t_lane + TM_QLO + 16 * j, lw);
+          for (int j = 0; j < 8; ++j) {
+            const uint4 x = valid ? src[8 * c + j] : make_uint4(0, 0, 0, 0);
+            v[4 * j + 0] = x.x; v[4 * j + 1] = x.y; v[4 * j + 2] = x.z; v[4 * j + 3] = x.w;
           }
-          tmem_st_wait();
-        } else {
-          const int sw = r_local & 7;
-#pragma unroll 2
-          for (int m = 0; m < 20; ++m) {   // features 256 + 16m .. +16
-            const uint4 x0 = valid ? src[32 + 2 * m] : z4, x1 = valid ? src[33 + 2 * m] : z4;
-            uint4 h, l;
-            f8_split8(x0, inv, h.x, h.y, l.x, l.y);
-            f8_split8(x1, inv, h.z, h.w, l.z, l.w);
-            uint8_t* hd;
-            uint8_t* ld;
-            int uh, ul;
-            if (m < 16) {
-              hd = qs_buf + (m >> 3) * F8_QS_CHUNK_BYTES;
-              ld = qs_buf + (2 + (m >> 3)) * F8_QS_CHUNK_BYTES;
-              uh = ul = m & 7;
-            } else {
-              hd = ld = qs_buf + 4 * F8_QS_CHUNK_BYTES;
-              uh = m - 16;
-              ul = m - 12;
-            }
-            *reinterpret_cast<uint4*>(hd + r_local * 128 + ((uh ^ sw) << 4)) = h;
-            *reinterpret_cast<uint4*>(ld + r_local * 128 + ((ul ^ sw) << 4)) = l;
-          }
-          fence_proxy_async_smem();
+          tmem_st32(tmem + t_lane + (hc ? TM_QLO : TM_QHI) + 32 * c, v);
         }
+        tmem_st_wait();
         tc_fence_before_sync();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.q_full);
