@@ -19,8 +19,9 @@
 //
 // Values. O_r = Σ_j P_rj C_j[:d_c] = Σ_j (P_rj sc_j) K_j[:d_c]: the scale joins P before P is
 // rounded to bf16, and the codes of this CTA's c_KV half are converted to bf16 in shared memory
-// (exactly: every E4M3 value is a bf16 value) by four converter warps, so P·C runs as in the
-// bf16 kernel. Rows outside the keys the unit sees are written as zeros there.
+// (exactly: every E4M3 value is a bf16 value), so P·C runs as in the bf16 kernel. The softmax
+// warps convert each tile right after agreeing on its row maxima, where they would otherwise
+// wait for the previous tile's P·C; rows outside the keys the unit sees are written as zeros.
 //
 // Shared memory: 2 stages x [4 code chunks of 64 tokens x 128 codes (128-byte swizzle) | k_R
 // codes 64 x 64 (64-byte swizzle)] = 36 KB each, 2 converted buffers of 4 x [64 x 64] bf16 (32 KB
@@ -29,8 +30,8 @@
 // the barriers. TMEM: [0,256) O half, [256,384) two score buffers, [384,448) hi and [448,512) lo
 // of the query's features 0..255 (four codes per column).
 //
-// Warp roles (448 threads): 0 TMA producer, 1 MMA issuer, 2..9 softmax (they also place each
-// unit's query features 0..255 in TMEM), 10..13 converters.
+// Warp roles (320 threads): 0 TMA producer, 1 MMA issuer, 2..9 softmax (they also place each
+// unit's query features 0..255 in TMEM and convert the value codes).
 #pragma once
 
 #include "fp8_cache.cuh"
@@ -46,15 +47,13 @@ constexpr int F8_STAGE_BYTES = 4 * F8_CHUNK_BYTES + F8_ROPE_BYTES;
 constexpr int F8_CV_BYTES = 4 * ATT_CHUNK_BYTES;                 // own c_KV half in bf16
 constexpr int F8_QS_CHUNKS = 5;
 constexpr int F8_QS_CHUNK_BYTES = 128 * 128;
-constexpr int F8_CONV_WARPS = 4;
-constexpr int F8_THREADS = 320 + 32 * F8_CONV_WARPS;
+constexpr int F8_THREADS = 320;
 constexpr uint32_t TM_QHI = TM_Q, TM_QLO = TM_Q + 64;
 
 struct AttnSharedF8 {
   float scales[ATT_STAGES][ATT_PAGE];   // the stage's token scales (bulk-copy target)
   uint64_t full_qk[ATT_STAGES], full_own[ATT_STAGES];
   uint64_t empty_qk[ATT_STAGES], empty_own[ATT_STAGES];
-  uint64_t cv_full[ATT_STAGES];        // converters wrote the stage's bf16 c_KV half
   uint64_t s_full[2], p_full[2], pv_done[2];
   uint64_t q_full;                     // the softmax warps placed a unit's query in TMEM
   uint64_t qs_full;                    // the unit's query chunks landed in shared memory (TMA)
@@ -171,6 +170,33 @@ qsplit_rows_kernel(const __nv_bfloat16* __restrict__ qhat, int n_rows, uint8_t* 
   if (lane == 0) alpha[row] = __fdiv_rn(am, E4M3_MAX_F);
 }
 
+// This CTA's c_KV half of a page, codes -> bf16 (exactly) in the K-major 128-byte-swizzled
+// chunks P·C reads ([64 tokens x 64 features] each), rows outside [z_lo, z_keep) written as
+// zeros: 1024 16-byte code units (source chunk j = i / 512, token row r, 16 features u), thread
+// tid of nthreads taking units tid, tid + nthreads, ...
+__device__ __forceinline__ void f8_convert_own(const uint8_t* src, uint8_t* dst, int tid,
+                                               int nthreads, int z_lo, int z_keep) {
+#pragma unroll 2
+  for (int i = tid; i < 1024; i += nthreads) {
+    const int j = i >> 9, r = (i >> 3) & 63, u = i & 7;
+    const int sw = r & 7;
+    uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
+    if (r >= z_lo && r < z_keep) {
+      const uint4 x = *reinterpret_cast<const uint4*>(src + j * F8_CHUNK_BYTES + r * 128 + ((u ^ sw) << 4));
+      e4m3x4_to_bf16x4(x.x, lo4.x, lo4.y);
+      e4m3x4_to_bf16x4(x.y, lo4.z, lo4.w);
+      e4m3x4_to_bf16x4(x.z, hi4.x, hi4.y);
+      e4m3x4_to_bf16x4(x.w, hi4.z, hi4.w);
+    }
+    // features 16u .. 16u+15 of source chunk j: bf16 chunk 2j + u/4, 16-byte units 2(u%4) and
+    // 2(u%4) + 1 of row r
+    uint8_t* d = dst + (2 * j + (u >> 2)) * ATT_CHUNK_BYTES + r * 128;
+    const int w0 = 2 * (u & 3);
+    *reinterpret_cast<uint4*>(d + ((w0 ^ sw) << 4)) = lo4;
+    *reinterpret_cast<uint4*>(d + (((w0 + 1) ^ sw) << 4)) = hi4;
+  }
+}
+
 // Score K-steps of one 128-code chunk c of a page into the score buffer at TMEM column d_s:
 // the hi and the lo part of the query each meet the chunk's four K = 32 steps. Chunks 0, 1
 // take A from TMEM, chunks 2, 3 from shared memory (query chunks c-2 (hi) and c (lo)).
@@ -221,7 +247,6 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       mbar_init(&sh.full_own[s], 1);
       mbar_init(&sh.empty_qk[s], 1);
       mbar_init(&sh.empty_own[s], 1);   // committed after the stage's P·C
-      mbar_init(&sh.cv_full[s], F8_CONV_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.s_full[b], 1);
@@ -353,7 +378,6 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
         const int st = gv % ATT_STAGES, sb = gv & 1;
         if (first_v && kv >= 1 && !att_warp_wait(sh, &sh.o_free, (kv - 1) & 1)) return false;
         if (!att_warp_wait(sh, &sh.p_full[sb], (gv >> 1) & 1)) return false;
-        if (!att_warp_wait(sh, &sh.cv_full[st], (gv / ATT_STAGES) & 1)) return false;
         tc_fence_after_sync();
         const uint64_t b0 = smem_desc_sw128(cv0 + st * F8_CV_BYTES, ATT_CHUNK_BYTES, 1024);
         mma_bf16_ts_mn_x4_elect(tmem + TM_O, tmem + TM_S + 64 * sb, b0, IDESC_PV, first_v ? 0u : 1u);
@@ -398,56 +422,6 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       mma_commit_elect(&sh.drain);
       if (lane == 0) (void)mbar_wait(&sh.drain, 0);
       __syncwarp();
-    } else if (warp >= 10) {
-      // ============================================================ converter warps
-      // This CTA's c_KV half of each page, codes -> bf16 in the K-major 128-byte-swizzled
-      // chunks P·C reads ([64 tokens x 64 features] each), rows outside the keys any row of the
-      // unit sees written as zeros. Thread ct takes 16-byte code units i = ct + 128k: source
-      // chunk j = i / 512, token row r, unit u (16 features).
-      const int ct = threadIdx.x - 320;
-      TileCursor cur;
-      cur.init(p.segs, seg_begin, seg_end);
-      int lo_u = 0, hi_u = -1;
-      for (int g = 0; cur.valid(); ++g, cur.next()) {
-        const int st = g % ATT_STAGES;
-        if (cur.first_of_seg()) {
-          const int b = cur.sg.unit / p.n_mt, mt = cur.sg.unit % p.n_mt;
-          const int L = p.seq_lens[b];
-          int unused;
-          visible_keys(p.keys, b, L, p.Tq, (mt * 128) / p.H, &lo_u, &unused);
-          visible_keys(p.keys, b, L, p.Tq, min(p.Tq - 1, (mt * 128 + 127) / p.H), &unused, &hi_u);
-        }
-        // the own chunks of tile g land only after P·C of tile g-2, which read this stage's
-        // converted buffer
-        if (!att_warp_wait(sh, &sh.full_own[st], (g / ATT_STAGES) & 1)) break;
-        const int z_lo = min(ATT_PAGE, max(0, lo_u - cur.tile * ATT_PAGE));
-        const int z_keep = max(z_lo, min(ATT_PAGE, hi_u + 1 - cur.tile * ATT_PAGE));
-        const uint8_t* src = stage_buf + st * F8_STAGE_BYTES + 2 * half * F8_CHUNK_BYTES;
-        uint8_t* dst = cv_buf + st * F8_CV_BYTES;
-#pragma unroll 2
-        for (int k = 0; k < 8; ++k) {
-          const int i = ct + 128 * k;
-          const int j = i >> 9, r = (i >> 3) & 63, u = i & 7;
-          const int sw = r & 7;
-          uint4 lo4 = make_uint4(0, 0, 0, 0), hi4 = make_uint4(0, 0, 0, 0);
-          if (r >= z_lo && r < z_keep) {
-            const uint4 x = *reinterpret_cast<const uint4*>(src + j * F8_CHUNK_BYTES + r * 128 + ((u ^ sw) << 4));
-            e4m3x4_to_bf16x4(x.x, lo4.x, lo4.y);
-            e4m3x4_to_bf16x4(x.y, lo4.z, lo4.w);
-            e4m3x4_to_bf16x4(x.z, hi4.x, hi4.y);
-            e4m3x4_to_bf16x4(x.w, hi4.z, hi4.w);
-          }
-          // features 16u .. 16u+15 of source chunk j: bf16 chunk 2j + u/4, 16-byte units
-          // 2(u%4) and 2(u%4) + 1 of row r
-          uint8_t* d = dst + (2 * j + (u >> 2)) * ATT_CHUNK_BYTES + r * 128;
-          const int w0 = 2 * (u & 3);
-          *reinterpret_cast<uint4*>(d + ((w0 ^ sw) << 4)) = lo4;
-          *reinterpret_cast<uint4*>(d + (((w0 + 1) ^ sw) << 4)) = hi4;
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.cv_full[st]);
-      }
     } else {
       // ============================================================ softmax warps
       const int hc = warp >= 6 ? 1 : 0;
@@ -498,8 +472,10 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
         const int L = p.seq_lens[b];
         const int r_in = mt * 128 + r_local;
         const bool row_valid = r_in < p.R;
-        int lo_row = 1, hi_row = 0;
+        int lo_row = 1, hi_row = 0, lo_u, hi_u, unused;
         if (row_valid) visible_keys(p.keys, b, L, p.Tq, r_in / p.H, &lo_row, &hi_row);
+        visible_keys(p.keys, b, L, p.Tq, (mt * 128) / p.H, &lo_u, &unused);
+        visible_keys(p.keys, b, L, p.Tq, min(p.Tq - 1, (mt * 128 + 127) / p.H), &unused, &hi_u);
         float m_ref = -INFINITY, l_part = 0.0f;
         for (int tile = sg.tile_begin; tile < sg.tile_end; ++tile, ++g) {
           const int sb = g & 1, st = g % ATT_STAGES;
@@ -543,6 +519,15 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           tc_fence_after_sync();
           const float raw_max = fmaxf(sh.row_max[g & 1][0][r_local], sh.row_max[g & 1][1][r_local]);
           const float mt_max = raw_max > -INFINITY ? raw_max * rowf : -INFINITY;
+          // this tile's c_KV half as bf16 for P·C (its codes have landed: S has read them; P·C
+          // of tile g-2, the last reader of this converted buffer, finished before S(g) began),
+          // done here, where the warps would otherwise wait for P·C of the previous tile
+          {
+            const int z_lo = min(ATT_PAGE, max(0, lo_u - tile * ATT_PAGE));
+            const int z_keep = max(z_lo, min(ATT_PAGE, hi_u + 1 - tile * ATT_PAGE));
+            f8_convert_own(stage_buf + st * F8_STAGE_BYTES + 2 * half * F8_CHUNK_BYTES,
+                           cv_buf + st * F8_CV_BYTES, hc * 128 + r_local, 256, z_lo, z_keep);
+          }
           float factor = 1.0f;
           bool rescale = false;
           if (mt_max > -INFINITY) {
@@ -601,6 +586,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           f2_unpack(ps2, ps0, ps1);
           l_part += ps0 + ps1;
           tmem_st_wait();
+          fence_proxy_async_smem();   // the converted half is read by P·C (async proxy)
           tc_fence_before_sync();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.p_full[sb]);
