@@ -246,7 +246,9 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
       mbar_init(&sh.full_qk[s], 1);
       mbar_init(&sh.full_own[s], 1);
       mbar_init(&sh.empty_qk[s], 1);
-      mbar_init(&sh.empty_own[s], 1);   // committed after the stage's P·C
+      // the stage's codes and scales are free once the score MMAs are done and the softmax
+      // warps have read the scales and converted the value codes: P·C reads the converted copy
+      mbar_init(&sh.empty_own[s], 1 + ATT_SM_WARPS);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sh.s_full[b], 1);
@@ -381,8 +383,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
         tc_fence_after_sync();
         const uint64_t b0 = smem_desc_sw128(cv0 + st * F8_CV_BYTES, ATT_CHUNK_BYTES, 1024);
         mma_bf16_ts_mn_x4_elect(tmem + TM_O, tmem + TM_S + 64 * sb, b0, IDESC_PV, first_v ? 0u : 1u);
-        mma_commit_elect(&sh.empty_own[st]);   // stage st (codes, scales, bf16 half) is free
-        mma_commit_elect(&sh.pv_done[sb]);
+        mma_commit_elect(&sh.pv_done[sb]);   // the score buffer and the converted half are free
         return true;
       };
       TileCursor cur;
@@ -413,6 +414,7 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
         f8_qk_chunk(tmem, d_s, b_stage, qs_desc, own, false);
         f8_qk_chunk(tmem, d_s, b_stage, qs_desc, own + 1, false);
         mma_commit_elect(&sh.s_full[sb]);
+        mma_commit_elect(&sh.empty_own[st]);   // the score MMAs are done with the codes
         if (cur.last_of_seg()) mma_commit_elect(&sh.q_free);
         if (g >= 1 && !issue_pv(g - 1, prev_first, prev_k)) { ok = false; break; }
         prev_first = cur.first_of_seg();
@@ -521,12 +523,15 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
           const float mt_max = raw_max > -INFINITY ? raw_max * rowf : -INFINITY;
           // this tile's c_KV half as bf16 for P·C (its codes have landed: S has read them; P·C
           // of tile g-2, the last reader of this converted buffer, finished before S(g) began),
-          // done here, where the warps would otherwise wait for P·C of the previous tile
+          // done here, where the warps would otherwise wait for P·C of the previous tile; the
+          // stage may then take the codes of tile g+2 while P·C of tile g is still to come
           {
             const int z_lo = min(ATT_PAGE, max(0, lo_u - tile * ATT_PAGE));
             const int z_keep = max(z_lo, min(ATT_PAGE, hi_u + 1 - tile * ATT_PAGE));
             f8_convert_own(stage_buf + st * F8_STAGE_BYTES + 2 * half * F8_CHUNK_BYTES,
                            cv_buf + st * F8_CV_BYTES, hc * 128 + r_local, 256, z_lo, z_keep);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.empty_own[st]);   // done with the codes and scales
           }
           float factor = 1.0f;
           bool rescale = false;
