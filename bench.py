@@ -176,6 +176,11 @@ def oracle_sample(w: WL.Workload, lens, pt, weights, cache_host, x_new, pos, q, 
     W_UK, W_UV = O.split_wkv_b(weights.wkv_b, w.H, w.d_nope, w.d_v)
     new_rows = O.latent_rows(x_new, weights.w_dkv, weights.kv_gain, pos.numpy(), w.d_c,
                              w.rms_eps, w.rope_theta)
+    if w.kv == "fp8":   # the stored rows: the new ones quantised, the history dequantised
+        new_rows = O.dequantize_rows_e4m3(*O.quantize_rows_e4m3(new_rows.astype("float32")))
+        n = WL.PAGE_SIZE * w.row
+        codes = cache_host[:, :n].view(cache_host.shape[0], WL.PAGE_SIZE, w.row).numpy()
+        scales = cache_host[:, n:].view(torch.float32).numpy()
     heads = [0, w.H // 2, w.H - 1, w.H // 3, (2 * w.H) // 3]
     done_units, done_work, elapsed = 0, 0, 0.0
     rows_cache = {}
@@ -186,7 +191,10 @@ def oracle_sample(w: WL.Workload, lens, pt, weights, cache_host, x_new, pos, q, 
         i += 1
         L = int(lens[b])
         if b not in rows_cache:
-            r = O.gather_rows(cache_host, pt.block_table[b].numpy(), L, WL.PAGE_SIZE)
+            if w.kv == "fp8":
+                r = O.gather_rows_fp8(codes, scales, pt.block_table[b].numpy(), L, WL.PAGE_SIZE)
+            else:
+                r = O.gather_rows(cache_host, pt.block_table[b].numpy(), L, WL.PAGE_SIZE)
             r[L - w.Tq:] = new_rows[b * w.Tq:(b + 1) * w.Tq]
             rows_cache = {b: r}
         t0 = time.perf_counter()
@@ -231,7 +239,7 @@ def run_reference(args, rank: int, world: int):
     """Reference arm: the fp64 oracle on this host's cores, same workload / metric / unit."""
     if rank != 0:
         return
-    w = WL.WORKLOADS[args.workload]
+    w = WL.get(args.workload)
     lens, pt, weights, cache_host, x_new, seq_idx, pos, q = build_inputs(w, "cpu")
     # each step: one (sequence, head) unit; the metric is total work / total time
     for _ in range(max(0, args.warmup)):

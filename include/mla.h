@@ -357,9 +357,10 @@ mla_status mla_prefill_ref(const mla_config* cfg, const void* x, const void* q, 
  * every GPU that loads the library holds until the process exits.
  *   - A call whose scratch need (mla_decode_workspace_size) exceeds that maximum returns
  *     MLA_ERR_WORKSPACE_TOO_SMALL and launches nothing. On a 148-SM B200, 32 MiB covers a
- *     DeepSeek-V2-shaped batch of up to 85 sequences with one query token each (the scratch
- *     holds Q̂ for every query row and one bf16 partial per split, whose count grows with the
- *     SM count).
+ *     DeepSeek-V2-shaped batch of up to 85 sequences with one query token each over a bf16
+ *     cache, 55 over a quantised one (the scratch holds Q̂ for every query row, with a
+ *     quantised cache also its split E4M3 form, and one bf16 partial per split, whose count
+ *     grows with the SM count).
  *   - It never calls cudaMalloc, cudaFree or any allocating routine.
  *   - The first call on a device looks up the array's device address (cudaGetSymbolAddress)
  *     and caches it; make that first call before any stream capture on that device.

@@ -65,3 +65,15 @@ def test_noalloc_rejects_a_batch_beyond_its_scratch():
         mla.mla_decode_noalloc(cfg, q, c.d["cache"], c.d["block_table"], c.d["seq_lens"],
                                c.d["w_uk_t"], c.d["w_uv"], out)
     assert e.value.code == 3   # MLA_ERR_WORKSPACE_TOO_SMALL, nothing launched
+
+
+def test_noalloc_decode_over_a_quantised_cache():
+    """The same built-in scratch serves a decode over an FP8 E4M3 cache (it then also holds the
+    split query rows): bit-identical to mla_decode on two calls in a row."""
+    mla.mla_get_device_error()
+    w = W.small_variant(V2, B=3, kv="fp8")
+    c = Hs.make_case(w, torch.tensor([1500, 64, 321], dtype=torch.int32))
+    Hs.run_append(c)
+    ref = Hs.run_decode(c).float().cpu()
+    for _ in range(2):
+        assert torch.equal(_noalloc(c), ref), "noalloc differs from mla_decode (quantised cache)"
