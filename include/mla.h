@@ -29,6 +29,8 @@
  *     stalled pipeline (a bounded wait that ran out, MLA_ERR_DEVICE_TIMEOUT) the kernel drains
  *     its copies and MMAs and leaves, and the call's outputs are undefined.
  *   - Calls that share a workspace or a cache must not overlap on the GPU (use one stream).
+ *   - Every call except mla_decode_noalloc opens an NVTX range named after it on the host
+ *     thread (visible to Nsight tools; a no-op without one).
  *   - Within a call, kernels after the first are launched with programmatic dependent launch
  *     and let the next kernel of the stream start early. A caller's own kernel enqueued right
  *     after a call with programmatic stream serialization must therefore wait
