@@ -88,3 +88,16 @@ def test_reference_arm_prints_one_json_line():
     assert d["impl"] == "reference" and d["value"] > 0 and d["unit"] == bench.UNIT
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_bench_accounts_for_the_quantised_cache():
+    """bench.py counts a quantised row as its codes plus one float32 scale, and one more
+    launch per step (the query split)."""
+    plain = bench.WL.get("v2_bf16_b64_ctx1kto32k_mix")
+    fp8 = bench.WL.get("v2_fp8_b64_ctx1kto32k_mix")
+    lens = torch.tensor([1000, 3000], dtype=torch.int32)
+    wp, wf = bench.work_of(plain, lens), bench.work_of(fp8, lens)
+    assert wp["cache_bytes"] == 4000 * 576 * 2
+    assert wf["cache_bytes"] == 4000 * (576 + 4)
+    assert wf["attn_flops"] == wp["attn_flops"] and wf["weight_bytes"] == wp["weight_bytes"]
+    assert bench.launches_per_step(plain) == 5 and bench.launches_per_step(fp8) == 6
