@@ -278,7 +278,6 @@ mla_decode_attn_fp8_kernel(const __grid_constant__ CUtensorMap map_c8,
   pdl_wait();
   pdl_trigger();
   const int seg_begin = p.pair_seg[pair], seg_end = p.pair_seg[pair + 1];
-  // the cache's first k_R row of a page sits 512 bytes into the page: map_r8 starts there
 
   if (seg_begin < seg_end) {
     if (warp == 0) {

@@ -7,7 +7,9 @@ through the C ABI, against the fp64 oracle.
 * The quantised append writes exactly the addressed slots; its rows dequantise to the oracle's
   rows within the E4M3 rounding bound.
 * Decode, prefill and partial decode over a quantised cache match the oracle run on the
-  dequantised rows (the oracle quantises its own new rows) within the bf16 parity bound.
+  dequantised rows (the oracle quantises its own new rows) within the bf16 parity bound,
+  including edge lengths, two query tokens, NaN-filled stale slots, the rescale path, a window,
+  full size and a cache of subnormal codes only.
 """
 
 import numpy as np
