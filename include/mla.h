@@ -195,7 +195,11 @@ size_t mla_decode_workspace_size(const mla_config* cfg, int32_t batch, int32_t t
  *   out         [batch, tq, n_heads, d_v]
  * bf16 runs on the tcgen05 tensor-core path and needs d_c = 512, d_rope = 64, page_size = 64
  * and d_nope a multiple of 64 (DeepSeek-V2 latent shapes); fp32 runs on CUDA cores for any
- * shape.
+ * shape. A quantised cache (kv_format MLA_KV_FP8_E4M3) runs on the tcgen05 path at the same
+ * shapes: the attention multiplies the E4M3 codes on the tensor cores (the query split into
+ * two E4M3 parts under a per-row scale, about 8 significant bits kept) and applies the
+ * per-token scales in the softmax; the result matches the same attention over the dequantised
+ * rows within the bf16 parity bound.
  * A sequence whose length is out of range gets zero output and MLA_ERR_DEVICE_BAD_LENGTH.
  */
 mla_status mla_decode(const mla_config* cfg, const void* q, int32_t batch, int32_t tq,
