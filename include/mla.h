@@ -13,11 +13,13 @@
  *
  * Conventions for every call:
  *   - Tensors are dense, row-major, and live in device memory unless stated otherwise. The
- *     element type of every floating-point tensor is cfg->dtype (fp32 or bf16). Index tensors
- *     are int32.
+ *     element type of every floating-point tensor is cfg->dtype (fp32 or bf16), except a
+ *     quantised cache (mla_kv_format below). Index tensors are int32.
  *   - The caller owns every buffer. The library never allocates or frees device memory and
  *     keeps no state between calls other than one device-side error word (see
- *     mla_get_device_error).
+ *     mla_get_device_error), the scratch array of mla_decode_noalloc, and a host-side cache of
+ *     encoded TMA descriptors (each a pure function of a tensor's address, shape and strides,
+ *     so a reused buffer skips re-encoding).
  *   - Device pointers must be 16-byte aligned.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream). Calls are asynchronous;
  *     they enqueue kernels on `stream` and return. Arguments are validated on the host first:
