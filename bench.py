@@ -593,6 +593,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             torch.cuda.empty_cache()
         line["other_workloads"] = extra
 
+    if world == 1 and not args.no_extra:
+        line["layer_calls"] = measure_layer_calls(mla, dev, flush_l2, min(K, 20))
+
     if rank == 0 and world == 1 and not args.no_cpu_baseline and w.kv == "plain":
         lens, pt, weights, cache_host, x_new_h, pos_h, q_h = cpu_case
         threading = ("serial loop over (sequence, head) units; cores = the BLAS thread count that "
@@ -609,6 +612,130 @@ def run_ours(args, rank: int, world: int, local_rank: int):
                                          "threading": threading}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def graph_time_ms(fn, flush_l2, K: int, dev) -> float:
+    """Mean device time of fn() over K calls captured in one CUDA graph, each after an L2 flush
+    that lies outside its events (3 eager warm-up calls first)."""
+    ev = lambda: torch.cuda.Event(enable_timing=True, external=True)
+    evs = [(ev(), ev()) for _ in range(K)]
+    for a, b in evs:
+        a.record()
+        b.record()
+    for i in range(3):
+        flush_l2(i)
+        fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(K):
+                flush_l2(i * 7)
+                evs[i][0].record()
+                fn()
+                evs[i][1].record()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    ms = statistics.fmean(a.elapsed_time(b) for a, b in evs)
+    del g
+    return ms
+
+
+def measure_layer_calls(mla, dev, flush_l2, K: int) -> dict:
+    """Device times of the layer's other calls at DeepSeek-V2 shape, each against its own
+    roofline: the q path and the output projection for the 16 query tokens of a batch-16
+    decode step (weight-streaming, HBM-bound), a tensor-core prefill of 2 prompts of 256 tokens
+    (tensor-bound) and a windowed decode (window 1024) of 16 sequences of 4096 tokens. Each
+    item is measured on its own; one that fails reports its error."""
+    pk, _ = peaks()
+    hbm, tc = float(pk["hbm_gbs"]), float(pk["bf16_tflops"])
+    bf = torch.bfloat16
+    res = {}
+    w = WL.get("v2_bf16_b16_ctx4096")
+    cfg = mla.make_config(w.H, w.d_model, w.d_c, w.d_r, w.d_nope, w.d_v, WL.PAGE_SIZE, w.dtype,
+                          w.scale, w.rms_eps, w.rope_theta)
+    n = w.B * w.Tq
+    try:
+        wt = WL.weights(w)
+        x = WL.randn((n, w.d_model), w.seed, 40, 1.0, bf).to(dev)
+        w_qa, q_gain, w_qb = wt.w_qa.to(dev), wt.q_gain.to(dev), wt.w_qb.to(dev)
+        q_out = torch.empty((n, w.H, w.d_nope + w.d_r), dtype=bf, device=dev)
+        ws = mla.workspace(mla.mla_query_workspace_size(cfg, w.q_lora, n), dev)
+        ms = graph_time_ms(lambda: mla.mla_query(cfg, x, w_qa, q_gain, w_qb, ws, q_out), flush_l2, K, dev)
+        nbytes = 2 * (w_qa.numel() + w_qb.numel() + x.numel() + q_out.numel())
+        res["query"] = {"what": f"mla_query, {n} tokens: wq_a, q_norm, wq_b", "ms_per_call": ms,
+                        "bound": "hbm", "algorithmic_bytes": nbytes,
+                        "roofline_frac": nbytes / (ms / 1e3) / 1e9 / hbm}
+        del wt, x, w_qa, q_gain, w_qb, q_out, ws
+    except Exception as e:
+        res["query"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        attn = WL.randn((n, w.H, w.d_v), w.seed, 41, 1.0, bf).to(dev)
+        w_o = WL.output_weight(w).to(dev)
+        y = torch.empty((n, w.d_model), dtype=bf, device=dev)
+        ws = mla.workspace(mla.mla_output_workspace_size(cfg, n), dev)
+        ms = graph_time_ms(lambda: mla.mla_output(cfg, attn, w_o, ws, y), flush_l2, K, dev)
+        nbytes = 2 * (w_o.numel() + attn.numel() + y.numel())
+        res["output"] = {"what": f"mla_output, {n} tokens: wo", "ms_per_call": ms, "bound": "hbm",
+                         "algorithmic_bytes": nbytes,
+                         "roofline_frac": nbytes / (ms / 1e3) / 1e9 / hbm}
+        del attn, w_o, y, ws
+    except Exception as e:
+        res["output"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        B, T = 2, 256
+        wp = WL.small_variant(WL.get("v2_bf16_b16_ctx4096"), B=B, Tq=T, lens=("fixed", T))
+        lens = WL.seq_lens(wp)
+        pt = WL.page_table(wp, lens)
+        wt = WL.weights(wp)
+        cache = WL.cache_pool(wp, pt.num_pages).to(dev)
+        x_new, _, _, q = WL.new_token_inputs(wp, lens)
+        x = x_new.view(B, T, wp.d_model).to(dev)
+        q = q.contiguous().to(dev)
+        w_uk_t = torch.empty((wp.H, wp.d_c, wp.d_nope), dtype=bf, device=dev)
+        w_uv = torch.empty((wp.H, wp.d_v, wp.d_c), dtype=bf, device=dev)
+        mla.mla_absorb_weights(cfg, wt.wkv_b.to(dev), w_uk_t, w_uv)
+        w_dkv, kv_gain = wt.w_dkv.to(dev), wt.kv_gain.to(dev)
+        bt, sl = pt.block_table.to(dev), lens.to(dev)
+        out = torch.empty((B, T, wp.H, wp.d_v), dtype=bf, device=dev)
+        ws = mla.workspace(mla.mla_prefill_workspace_size(cfg, B, T), dev)
+        ms = graph_time_ms(lambda: mla.mla_prefill(cfg, x, q, w_dkv, kv_gain, w_uk_t, w_uv, sl, bt,
+                                                   cache, ws, out), flush_l2, K, dev)
+        n_tok = B * T
+        flops = (wp.H * 2 * (wp.row + wp.d_c) * B * T * (T + 1) // 2     # causal attention
+                 + 2 * n_tok * wp.row * wp.d_model                         # down-projection
+                 + 2 * 2 * n_tok * wp.H * wp.d_nope * wp.d_c)              # W_UK and W_UV
+        res["prefill"] = {"what": f"mla_prefill, {B} prompts of {T} tokens (append, absorbed "
+                                  "query, causal latent attention, W_UV)",
+                          "ms_per_call": ms, "prompt_tokens_per_s": n_tok / (ms / 1e3),
+                          "bound": "tensor", "algorithmic_flops": flops,
+                          "roofline_frac": flops / (ms / 1e3) / 1e12 / tc}
+        del cache, x, q, w_uk_t, w_uv, w_dkv, kv_gain, bt, sl, out, ws, wt
+    except Exception as e:
+        res["prefill"] = {"error": f"{type(e).__name__}: {e}"}
+    try:
+        ww = WL.get("v2_bf16_b16_ctx4096")
+        cw = DeviceCase(mla, ww, dev)
+        cw.cfg.window = 1024
+        mla.mla_append_latent(cw.cfg, cw.x_new, cw.w_dkv, cw.kv_gain, cw.seq_idx, cw.pos, cw.bt,
+                              cw.cache, cw.ws_a)
+        ms = graph_time_ms(cw.decode, flush_l2, K, dev)
+        keys = sum(min(int(L), 1024) for L in cw.lens.tolist())
+        nbytes = keys * ww.row * 2
+        res["window_decode"] = {"what": "mla_decode, 16 sequences of 4096 tokens, window 1024",
+                                "ms_per_call": ms,
+                                "value": keys * ww.Tq * ww.H / (ms / 1e3), "unit": UNIT,
+                                "bound": "hbm", "algorithmic_bytes": nbytes + cw.work["weight_bytes"],
+                                "roofline_frac": (nbytes + cw.work["weight_bytes"]) / (ms / 1e3) / 1e9 / hbm}
+        del cw
+    except Exception as e:
+        res["window_decode"] = {"error": f"{type(e).__name__}: {e}"}
+    torch.cuda.empty_cache()
+    return res
 
 
 def stored_traffic(workload: str):
